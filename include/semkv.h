@@ -1,0 +1,217 @@
+/*
+ * semkv.h -- C ABI of the SemKV mixed-precision KV-cache hot path (libsemkv.so).
+ *
+ * The method: "SemKV: Semantic Mixed-Precision KV Cache Quantization Guided by
+ * the Quality Cliff for Long-Context LLM Inference" (D. Lee, D.-H. Kim,
+ * J.-H. Kim).  Every prompt token is scored by one model-internal indicator
+ * (Fig. 2), tokens are ranked within the prompt and the top r get the high
+ * level count, the rest the adjacent low one (Fig. 4); the per-token choice is
+ * broadcast over every layer and KV head, for K and V alike (Fig. 5); each row
+ * of head_dim values is affine-quantized (Table 2, Table 6: two scalars per
+ * row); generated tokens wait in an FP16 block that is ranked and quantized as
+ * a whole when it fills (Fig. 6); decoding attends over the mixed cache
+ * (Fig. 5).
+ *
+ * Conventions for every call
+ *   - Tensor pointers are DEVICE pointers owned by the caller.  The library
+ *     never allocates, frees or synchronizes; every call only enqueues work on
+ *     `stream` (a cudaStream_t passed as void*, NULL = legacy default stream).
+ *   - fp16 tensors are IEEE binary16 bit patterns (uint16_t), fp32 is IEEE
+ *     binary32.  KV tensors are laid out [B][n_layers][H][T][D] (row = D values).
+ *   - Every tensor pointer must be 16-byte aligned.
+ *   - Arguments are validated on the host before anything is launched; a bad
+ *     argument returns an error and enqueues nothing.
+ *   - Conditions only the GPU can see (a non-finite input, a pool that would
+ *     overflow, a length beyond T_max) are OR-ed as SEMKV_FLAG_* bits into the
+ *     caller's device word `status` (may be NULL for calls that take none);
+ *     the caller reads it after synchronizing.  Kernels never trap and never
+ *     spin-wait.
+ *   - D (head_dim) must be 128; level counts L must be in [2, 16].
+ */
+#ifndef SEMKV_H
+#define SEMKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum semkv_status {
+  SEMKV_OK = 0,
+  SEMKV_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape    */
+  SEMKV_ERR_UNSUPPORTED = 2,   /* D != 128, L outside [2,16], H_q/H > 8          */
+  SEMKV_ERR_WORKSPACE = 3,     /* workspace smaller than the *_workspace_size    */
+  SEMKV_ERR_CAPACITY = 4,      /* an append would overflow the FP16 block        */
+  SEMKV_ERR_CUDA = 5           /* a launch failed (cudaGetLastError)             */
+} semkv_status;
+
+/* device status bits (OR-ed into *status) */
+#define SEMKV_FLAG_NONFINITE 0x1u  /* a quantized row or a score held NaN/Inf; that row's output is unspecified */
+#define SEMKV_FLAG_CAPACITY  0x2u  /* a row did not fit its pool; it was not written                           */
+#define SEMKV_FLAG_SEQLEN    0x4u  /* seq_len[b] outside [0, T_max]; the sequence was skipped                  */
+
+typedef enum semkv_score_kind {
+  SEMKV_SCORE_ATTN_MASS = 0,   /* attention mass from the last w query rows (Table 1 "Attn."; Fig. 10) */
+  SEMKV_SCORE_KEY_L2 = 1       /* key L2 norm over the scoring layer's KV heads (Table 3 "key-norm")   */
+} semkv_score_kind;
+
+#define SEMKV_FLUSH 0x1u       /* semkv_append_block: quantize the partial FP16 block (end of turn, Fig. 6) */
+
+/*
+ * The mixed cache.  A host-side struct of sizes and device pointers; the pools
+ * are caller-allocated device memory of the sizes given below.  Pool layout
+ * per class c in {high, low}, with W_c = semkv_words_per_row(L_c, 128):
+ *   codes  k_c, v_c : uint32 [B][n_layers][H][cap_c][W_c]   mixed-radix words
+ *   meta   k_c_meta, v_c_meta : float [B][n_layers][H][cap_c][2] = (min, scale)
+ * Within a (sequence, layer, head) a class keeps its tokens in token order:
+ * slot = number of same-class tokens quantized before it.  n_high[b] and
+ * n_low[b] (device int32) count the slots in use; they are the same for every
+ * layer and head because the token-wise choice is broadcast (Fig. 5).
+ * The FP16 block (Fig. 6): buf_k, buf_v fp16 [B][n_layers][H][block][128],
+ * buf_score fp32 [B][block]; buf_len (HOST field) tokens of it are in use,
+ * the same number for every sequence.
+ */
+typedef struct semkv_cache {
+  int32_t B, n_layers, H, H_q, D;
+  int32_t L_high, L_low;
+  int32_t r_ppm;                 /* high fraction r in parts per million, [0, 1e6]   */
+  int32_t cap_high, cap_low;     /* slots per (sequence, layer, head); multiples of 16 */
+  int32_t block;                 /* FP16 block length (128)                          */
+  int32_t buf_len;               /* host: tokens in the FP16 block, 0 <= buf_len < block */
+  uint32_t *k_high, *v_high, *k_low, *v_low;
+  float *k_high_meta, *v_high_meta, *k_low_meta, *v_low_meta;
+  int32_t *n_high, *n_low;       /* device [B] */
+  uint16_t *buf_k, *buf_v;       /* device fp16 [B][n_layers][H][block][D] */
+  float *buf_score;              /* device [B][block] */
+} semkv_cache;
+
+/* ---- host helpers (no GPU work) ------------------------------------------ */
+
+/* ceil(r * n) with r = r_ppm / 1e6, exact in integers (Fig. 4: exactly the top r).
+ * Returns -1 if n < 0 or r_ppm is outside [0, 1e6]. */
+int64_t semkv_num_high(int64_t n, int32_t r_ppm);
+
+/* Base-L digits per 32-bit word: the largest n with L^n <= 2^32, i.e.
+ * floor(32 / log2 L) (Fig. 1: L levels carry log2 L bits).  -1 if L not in [2,16]. */
+int32_t semkv_digits_per_word(int32_t L);
+
+/* 32-bit words per row of D codes: ceil(D / digits_per_word(L)); -1 if invalid. */
+int32_t semkv_words_per_row(int32_t L, int32_t D);
+
+/* Library build identification string (static storage). */
+const char *semkv_version(void);
+
+/* ---- a1: importance score (Fig. 2) ---------------------------------------- */
+
+/* Workspace bytes semkv_score needs for these sizes (0 for KEY_L2). */
+size_t semkv_score_workspace_size(int32_t kind, int32_t B, int32_t T_max, int32_t H,
+                                  int32_t H_q, int32_t w);
+
+/*
+ * Per-token importance score of one scoring layer.
+ *   k       fp16, sequence b's keys at k + b*k_batch_stride, laid out [H][T_max][D]
+ *           (so a [B][n_layers][H][T_max][D] cache passes its layer slice with
+ *           k_batch_stride = n_layers*H*T_max*D).
+ *   q_win   fp16 [B][H_q][w][D]: the last w query rows of the scoring layer
+ *           (ATTN_MASS only; NULL for KEY_L2).  Row i sits at position
+ *           seq_len[b] - w + i and sees keys j <= that position; rows whose
+ *           position is negative are skipped.  Query head h reads KV head
+ *           floor(h / (H_q/H)); logits are scaled by 1/sqrt(D).
+ *   seq_len int32 [B], tokens of each sequence (<= T_max).
+ *   score   fp32 [B][T_max]; entries j >= seq_len[b] are written 0.
+ * ATTN_MASS: s_j = sum_h sum_i softmax_j(q_hi . k_j / sqrt(D)) (fp32 tensor-core
+ *   products, fp32 softmax; within 1e-4 relative of the float64 definition).
+ * KEY_L2: s_j = sqrt(sum over heads and dims of k^2), in one fixed fp32 order:
+ *   per head, 32 lane partials (x0^2+x1^2)+(x2^2+x3^2) over dims 4l..4l+3,
+ *   an xor butterfly over 16,8,4,2,1, then heads summed in order, IEEE sqrt.
+ * Errors: INVALID_ARG (null/misaligned, B,T_max,H <= 0, H_q % H, w <= 0),
+ * UNSUPPORTED (D != 128, H_q/H > 8), WORKSPACE.
+ */
+semkv_status semkv_score(int32_t kind, const uint16_t *k, int64_t k_batch_stride,
+                         const uint16_t *q_win, const int32_t *seq_len, int32_t B,
+                         int32_t T_max, int32_t H, int32_t H_q, int32_t D, int32_t w,
+                         float *score, void *ws, size_t ws_bytes, uint32_t *status,
+                         void *stream);
+
+/* ---- a2: per-prompt top-r selection (Fig. 2, Fig. 4) ---------------------- */
+
+size_t semkv_select_workspace_size(int32_t B, int32_t T_max);
+
+/*
+ * mask[b][j] = 1 for the first ceil(r*seq_len[b]) tokens of sequence b in the
+ * order (score descending, token index ascending), else 0; -0.0 ranks as +0.0.
+ * No threshold is estimated: exactly that many tokens are high (Fig. 4), and
+ * every other token is low, none is dropped (Table 1).
+ *   score fp32 [B][T_max]; mask uint8 [B][T_max] (entries >= seq_len[b] set 0).
+ *   seq_len int32 [B] (device), or NULL to use len_const for every sequence.
+ * A NaN score sets SEMKV_FLAG_NONFINITE (the mask is then unspecified).
+ */
+semkv_status semkv_select(const float *score, int64_t score_batch_stride,
+                          const int32_t *seq_len, int32_t len_const, int32_t B,
+                          int32_t T_max, int32_t r_ppm, uint8_t *mask,
+                          int64_t mask_batch_stride, void *ws, size_t ws_bytes,
+                          uint32_t *status, void *stream);
+
+/* ---- a3+a4: quantize and pack into the pools (Fig. 5; Table 2; Table 6) ---- */
+
+size_t semkv_quantize_workspace_size(int32_t B, int32_t T_max);
+
+/*
+ * Quantize every row of K and V [B][n_layers][H][T_max][D] (fp16) with tokens
+ * j < seq_len[b], row class from mask[b][j] (1 = high), and append the rows to
+ * the pools after the slots already in use (n_high[b], n_low[b]), which are
+ * then advanced.  Per row, in IEEE fp32 round-to-nearest-even:
+ *   mn = min(x)+0, mx = max(x)+0, scale = (mx-mn)/(L-1),
+ *   code = scale == 0 ? 0 : clamp(rint((x-mn)/scale), 0, L-1)      (exact division)
+ *   word w = sum_j code[w*n+j] * L^j, n = semkv_digits_per_word(L)  (little-endian digits)
+ *   meta = (mn, scale).
+ * Bit-identical to the definition for all finite inputs.  Rows beyond a pool's
+ * capacity are not written (SEMKV_FLAG_CAPACITY); non-finite rows set
+ * SEMKV_FLAG_NONFINITE.
+ */
+semkv_status semkv_quantize(semkv_cache *c, const uint16_t *k, const uint16_t *v,
+                            int32_t T_max, const int32_t *seq_len, const uint8_t *mask,
+                            void *ws, size_t ws_bytes, uint32_t *status, void *stream);
+
+/* ---- a5: generation-time block-exact path (Fig. 6) ------------------------- */
+
+size_t semkv_append_workspace_size(const semkv_cache *c);
+
+/*
+ * Append n new tokens per sequence: k_new, v_new fp16 [B][n_layers][H][n][D],
+ * score_new fp32 [B][n] (any indicator; only its ranking within a block is used).
+ * Tokens go to the FP16 block; each time it holds `block` tokens, its own
+ * scores are ranked, the top ceil(r*block) get L_high, the block is quantized
+ * onto the pools exactly as semkv_quantize does, and emptied.  A full block is
+ * never left in FP16.  flags & SEMKV_FLUSH (end of a generation turn): after
+ * appending, a partial block of m > 0 tokens is quantized the same way with
+ * ceil(r*m) high tokens.  Updates c->buf_len on the host.  n may be 0.
+ */
+semkv_status semkv_append_block(semkv_cache *c, const uint16_t *k_new, const uint16_t *v_new,
+                                const float *score_new, int32_t n, uint32_t flags, void *ws,
+                                size_t ws_bytes, uint32_t *status, void *stream);
+
+/* ---- a6: decode attention over the mixed cache (Fig. 5) -------------------- */
+
+size_t semkv_decode_workspace_size(const semkv_cache *c, int32_t n_layers);
+
+/*
+ * One decode query per query head for layers [layer0, layer0+n_layers):
+ *   q   fp16 [B][n_layers][H_q][D];  out fp16 [B][n_layers][H_q][D].
+ * out_h = sum_j softmax_j(sm_scale * q_h . k_j) v_j over every cached token of
+ * KV head floor(h/(H_q/H)): the high pool, the low pool (dequantized as
+ * mn + code*scale) and the buf_len FP16 tokens.  A sequence with no cached
+ * token gets out = 0.  fp32 softmax, fp16 tensor-core products: within 1e-3
+ * relative L2 of the float64 definition.
+ */
+semkv_status semkv_decode_attn(const semkv_cache *c, int32_t layer0, int32_t n_layers,
+                               const uint16_t *q, uint16_t *out, float sm_scale, void *ws,
+                               size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SEMKV_H */

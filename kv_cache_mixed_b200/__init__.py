@@ -1,0 +1,10 @@
+"""SemKV token-wise mixed-precision KV-cache hot path for B200 (sm_100a).
+
+The kernels live in libsemkv.so (C ABI: include/semkv.h); this package is a
+thin binding with the same names.  Importing it fails loudly if the library
+has not been built (`python -m kv_cache_mixed_b200.build`).
+"""
+from .binding import (FLAG_CAPACITY, FLAG_NONFINITE, FLAG_SEQLEN, FLUSH, SCORE_ATTN_MASS,  # noqa: F401
+                      SCORE_KEY_L2, EXPORTED, LIB_PATH, MixedCache, SemkvError, semkv_append_block,
+                      semkv_decode_attn, semkv_digits_per_word, semkv_num_high, semkv_quantize,
+                      semkv_score, semkv_select, semkv_version, semkv_words_per_row)

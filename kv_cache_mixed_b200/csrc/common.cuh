@@ -1,0 +1,132 @@
+// common.cuh -- shared device helpers of libsemkv (sm_100a).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/semkv.h"
+
+namespace semkv {
+
+constexpr int kD = 128;          // head_dim
+constexpr int kMaxL = 16;
+
+// ---------------------------------------------------------------------------
+// Layout sizes (compile-time twins of semkv_digits_per_word / words_per_row)
+// ---------------------------------------------------------------------------
+__host__ __device__ constexpr int digits_per_word(int L) {
+  // largest n with L^n <= 2^32
+  int n = 0;
+  unsigned long long p = 1;
+  while (p * (unsigned long long)L <= (1ull << 32)) {
+    p *= (unsigned long long)L;
+    ++n;
+  }
+  return n;
+}
+__host__ __device__ constexpr int words_per_row(int L) {
+  return (kD + digits_per_word(L) - 1) / digits_per_word(L);
+}
+__host__ __device__ constexpr unsigned long long ipow(int L, int k) {
+  unsigned long long p = 1;
+  for (int i = 0; i < k; ++i) p *= (unsigned long long)L;
+  return p;
+}
+
+// ---------------------------------------------------------------------------
+// Device status word
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void set_flag(uint32_t *status, uint32_t f) {
+  if (status) atomicOr(status, f);
+}
+
+// ---------------------------------------------------------------------------
+// Fast unsigned division by a runtime constant (Granlund-Montgomery style
+// multiply-high + shift).  Valid for numerators < 2^31 and divisors >= 1.
+// ---------------------------------------------------------------------------
+struct FastDiv {
+  uint32_t d, m, s;
+  __host__ FastDiv() : d(1), m(0), s(0) {}
+  __host__ explicit FastDiv(uint32_t div) : d(div) {
+    // smallest s with 2^s >= d; m = floor(2^(32+s) / d) + 1 - 2^32 (the
+    // classic round-up reciprocal for 31-bit numerators)
+    s = 0;
+    while ((1ull << s) < d) ++s;
+    unsigned long long mm = ((1ull << (32 + s)) + d - 1) / d;   // ceil(2^(32+s)/d)
+    m = (uint32_t)(mm - (1ull << 32));
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    uint32_t t = __umulhi(n, m);
+    return (t + n) >> s;    // n < 2^31 so t + n does not overflow
+  }
+};
+
+// ---------------------------------------------------------------------------
+// Small PTX wrappers (documented instructions only)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;\n" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint4 ld_stream_u4(const void *p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
+}
+
+// max that propagates NaN (PTX max.NaN, sm_80+)
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
+__device__ __forceinline__ float ex2_approx(float x) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// D = A(16x16, f16, row) * B(16x8, f16, col) + C, fp32 accumulate
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};\n"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// transpose of an 8x8 b16 matrix held one row-pair per lane
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t r;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;\n" : "=r"(r) : "r"(x));
+  return r;
+}
+
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], const void *smem) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(smem)));
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  __half2 h = __floats2half2_rn(lo, hi);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+}  // namespace semkv

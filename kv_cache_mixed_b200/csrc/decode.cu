@@ -1,0 +1,562 @@
+// decode.cu -- GQA decode attention over the mixed-precision cache (SemKV,
+// Fig. 5: "the mixed-precision quantized KV cache used for decoding"; Fig. 6:
+// the most recent partial block stays FP16 during decoding).
+//
+// Attention works in the code domain, so no row is ever dequantized:
+//   q . khat_j = scale_j * (q . c_j) + mn_j * sum(q)
+//   sum_j p_j vhat_j = sum_j (p_j scale_j) c_j + (sum_j p_j mn_j) * 1
+// Both dot products run on tensor cores (mma.sync m16n8k16, f16 x f16 -> f32).
+// Codes enter the tensor cores as raw f16 subnormal bit patterns c * 2^-24
+// (exact), so a digit costs no conversion: unpacking a 32-bit word gives the
+// digit in the low bits of a register and two digits packed in one register
+// are already an f16x2 operand.  The 2^24 factor is folded into the scales.
+//
+// Digit extraction (any L in [2,16]): a word is split by constant divisors into
+// parts of k digits with L^k small enough that, with F = v * ceil(2^32/L^k),
+// each step t = F * L yields the next digit (most significant first) in the
+// high 32 bits and the next F in the low 32 bits.  The part sizes below were
+// checked exhaustively against repeated division for every part value.
+//
+// Work split: one pool class per launch (template on its L); CTA = 4 warps on
+// a contiguous range of 16-token tiles of one (sequence, layer, KV head); each
+// warp streams its tiles through a cp.async ring in shared memory; online
+// softmax in the log2 domain; the 4 warps merge in shared memory and the CTA
+// writes one partial (m, l, o[128]) per query head.  The FP16 block gets its
+// own small kernel and a last kernel merges all partials of a (sequence,
+// layer, KV head) into the output.
+#include "common.cuh"
+#include "internal.h"
+
+namespace semkv {
+
+constexpr int DEC_WARPS = 4;
+constexpr int DEC_NST = 4;                  // tiles in flight per warp
+constexpr int DEC_GMAX = 8;                 // query heads per KV head handled (M rows used)
+constexpr int PART_STRIDE = 132;            // floats per partial: m, l, pad, pad, o[128]
+constexpr float kLog2eF = 1.4426950408889634f;
+
+// ---- digit split table: part sizes in digits, least significant part first
+__host__ __device__ constexpr int split_part(int L, int i) {
+  // {part0, part1, part2} per L; a 0 marks an unused part
+  return L == 2 ? (i < 2 ? 16 : 0) : L == 3 ? (i < 2 ? 10 : 0) : L == 4 ? (i < 2 ? 8 : 0)
+       : L == 5 ? (i == 0 ? 6 : i == 1 ? 7 : 0) : L == 6 ? (i < 2 ? 6 : 0)
+       : L == 7 ? (i == 0 ? 3 : 4) : L == 8 ? (i < 2 ? 5 : 0) : L == 9 ? (i < 2 ? 5 : 0)
+       : L == 10 ? (i == 0 ? 4 : i == 1 ? 5 : 0) : L == 11 ? 3 : (i < 2 ? 4 : 0);
+}
+__host__ __device__ constexpr int split_parts(int L) { return (L == 7 || L == 11) ? 3 : 2; }
+
+template <int L>
+struct Geo {
+  static constexpr int N = digits_per_word(L);       // digits per word
+  static constexpr int W = words_per_row(L);         // words per row
+  static constexpr int WPG = (W + 3) / 4;            // words per lane group (lane % 4)
+  static constexpr int KB = (WPG * N + 3) / 4;       // 16-slot k-blocks
+  static constexpr int TILE_BYTES = 16 * W * 4 * 2 + 16 * 8 * 2;
+  static_assert(split_part(L, 0) + split_part(L, 1) + split_part(L, 2) == N, "split must cover the word");
+};
+
+// digit j (0 = least significant) of word w into dig[j0 + j]
+template <int L, int NDIG>
+__device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&dig)[NDIG], int j0) {
+  constexpr int NP = split_parts(L);
+  uint32_t rest = w;
+  int jb = j0;
+#pragma unroll
+  for (int pi = 0; pi < NP; ++pi) {
+    const int k = split_part(L, pi);
+    uint32_t v;
+    if (pi < NP - 1) {
+      const uint32_t P = (uint32_t)ipow(L, k);
+      const uint32_t qq = rest / P;
+      v = rest - qq * P;
+      rest = qq;
+    } else {
+      v = rest;
+    }
+    const uint32_t M = (uint32_t)(((1ull << 32) + ipow(L, k) - 1) / ipow(L, k));
+    uint32_t F = v * M;
+#pragma unroll
+    for (int d = k - 1; d >= 0; --d) {
+      const unsigned long long t = (unsigned long long)F * (unsigned long long)L;
+      dig[jb + d] = (uint32_t)(t >> 32);
+      F = (uint32_t)t;
+    }
+    jb += k;
+  }
+}
+
+// The lane group c = lane % 4 owns words c*WPG .. c*WPG+WPG-1 of a token row.
+// Its digit slot u = i*N + j (word i, digit j) sits in k-block u/4 at
+// position u%4; positions 0,1 are one f16x2 register, 2,3 the other.
+template <int L>
+__device__ __forceinline__ void unpack_row(const uint32_t *wrow, int c,
+                                           uint32_t (&reg)[Geo<L>::KB][2]) {
+  using G = Geo<L>;
+  constexpr int ND = G::KB * 4;
+  uint32_t dig[ND];
+#pragma unroll
+  for (int i = 0; i < G::WPG; ++i) {
+    const int wi = c * G::WPG + i;
+    const uint32_t w = wi < G::W ? wrow[wi] : 0u;
+    extract_word<L, ND>(w, dig, i * G::N);
+  }
+#pragma unroll
+  for (int u = G::WPG * G::N; u < ND; ++u) dig[u] = 0u;
+#pragma unroll
+  for (int kb = 0; kb < G::KB; ++kb) {
+    reg[kb][0] = dig[4 * kb] | (dig[4 * kb + 1] << 16);
+    reg[kb][1] = dig[4 * kb + 2] | (dig[4 * kb + 3] << 16);
+  }
+}
+
+// head-dim index of slot u of lane group c (or -1 for a padding slot)
+template <int L>
+__device__ __forceinline__ int slot_dim(int c, int u) {
+  using G = Geo<L>;
+  const int wi = c * G::WPG + u / G::N;
+  const int d = wi * G::N + u % G::N;
+  return (u < G::WPG * G::N && wi < G::W && d < kD) ? d : -1;
+}
+
+struct DecParams {
+  // pool of this launch
+  const uint32_t *kw, *vw;          // [B][Lyr][H][cap][W]
+  const float2 *km, *vm;            // [B][Lyr][H][cap]
+  const int32_t *count;             // [B]
+  int cap;
+  // cache geometry
+  int B, Lyr, H, H_q, G, layer0, nL;
+  const uint16_t *q;                // [B][nL][H_q][D]
+  float c2;                         // sm_scale * log2(e)
+  float *part;                      // [slabs][NU][G][PART_STRIDE]
+  int NU, unit0, S;                 // units per slab, first unit of this launch, splits
+};
+
+constexpr int kMergeBytes = DEC_WARPS * DEC_GMAX * kD * 4 + DEC_WARPS * DEC_GMAX * 3 * 4;
+template <int L>
+constexpr int kQOff = (DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES > kMergeBytes)
+                          ? DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES : kMergeBytes;
+
+template <int L>
+__global__ void __launch_bounds__(DEC_WARPS * 32)
+decode_pool_kernel(const DecParams p) {
+  using Gm = Geo<L>;
+  constexpr int KB = Gm::KB, W = Gm::W;
+  constexpr float kappa = (L == 2) ? 0.5f : 1.0f;       // keeps p*scale inside f16 range
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
+  const int slab = blockIdx.x / p.S, split = blockIdx.x % p.S;
+  const int h = slab % p.H, li = (slab / p.H) % p.nL, b = slab / (p.H * p.nL);
+  const int64_t pslab = ((int64_t)b * p.Lyr + p.layer0 + li) * p.H + h;
+  const int G = p.G;
+
+  // ---- shared memory: per-warp tile rings, then the q rows
+  uint8_t *ring = smem + warp * DEC_NST * Gm::TILE_BYTES;
+  float *qs = reinterpret_cast<float *>(smem + kQOff<L>);   // [G][128]
+  for (int i = threadIdx.x; i < G * kD; i += DEC_WARPS * 32) {
+    const int qh = i / kD, d = i % kD;
+    const uint16_t hb = p.q[(((int64_t)b * p.nL + li) * p.H_q + h * G + qh) * kD + d];
+    qs[i] = __half2float(__ushort_as_half(hb));
+  }
+  __syncthreads();
+
+  // ---- q fragments in slot order, and sum(q) * c2 for this lane's query r
+  uint32_t qa[KB][2];
+  float qsum = 0.0f;
+#pragma unroll
+  for (int kb = 0; kb < KB; ++kb) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      float v[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int d = slot_dim<L>(c, 4 * kb + 2 * hh + e);
+        v[e] = (r < G && d >= 0) ? qs[r * kD + d] : 0.0f;
+        qsum += v[e];
+      }
+      qa[kb][hh] = pack_half2(v[0], v[1]);
+    }
+  }
+  qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
+  qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
+  const float qsc = qsum * p.c2;
+  const float kscale = p.c2 * 16777216.0f;             // 2^24: codes are c * 2^-24
+
+  // ---- this CTA's tiles
+  const int n = min(p.count[b], p.cap);
+  const int ntile = (n + 15) >> 4;
+  const int tb = (int)((int64_t)ntile * split / p.S), te = (int)((int64_t)ntile * (split + 1) / p.S);
+  const uint32_t *kw = p.kw + pslab * p.cap * W;
+  const uint32_t *vw = p.vw + pslab * p.cap * W;
+  const float2 *km = p.km + pslab * p.cap;
+  const float2 *vm = p.vm + pslab * p.cap;
+
+  auto issue = [&](int tile, int slotix) {
+    if (tile < te) {
+      uint8_t *dst = ring + slotix * Gm::TILE_BYTES;
+      const int t0 = tile * 16;
+      const uint8_t *kwb = reinterpret_cast<const uint8_t *>(kw + (int64_t)t0 * W);
+      const uint8_t *vwb = reinterpret_cast<const uint8_t *>(vw + (int64_t)t0 * W);
+      const uint8_t *kmb = reinterpret_cast<const uint8_t *>(km + t0);
+      const uint8_t *vmb = reinterpret_cast<const uint8_t *>(vm + t0);
+      constexpr int ch_w = 4 * W;           // 16-byte chunks of one 16-token word block
+      constexpr int total = 2 * ch_w + 16;
+      for (int i = lane; i < total; i += 32) {
+        const uint8_t *src;
+        int doff;
+        if (i < ch_w) { src = kwb + i * 16; doff = i * 16; }
+        else if (i < 2 * ch_w) { src = vwb + (i - ch_w) * 16; doff = i * 16; }
+        else if (i < 2 * ch_w + 8) { src = kmb + (i - 2 * ch_w) * 16; doff = i * 16; }
+        else { src = vmb + (i - 2 * ch_w - 8) * 16; doff = i * 16; }
+        cp_async16(dst + doff, src);
+      }
+    }
+    cp_async_commit();
+  };
+
+  float m_run = -INFINITY, l_run = 0.0f, mt_run = 0.0f;
+  float oacc[KB][4];
+#pragma unroll
+  for (int kb = 0; kb < KB; ++kb) oacc[kb][0] = oacc[kb][1] = oacc[kb][2] = oacc[kb][3] = 0.0f;
+
+  // ring prologue
+  int next = tb + warp;
+#pragma unroll
+  for (int s = 0; s < DEC_NST - 1; ++s) {
+    issue(next, s);
+    next += DEC_WARPS;
+  }
+  int slotix = 0;
+  for (int tile = tb + warp; tile < te; tile += DEC_WARPS) {
+    issue(next, (slotix + DEC_NST - 1) % DEC_NST);
+    next += DEC_WARPS;
+    cp_async_wait<DEC_NST - 1>();
+    __syncwarp();
+    const uint8_t *tbuf = ring + slotix * Gm::TILE_BYTES;
+    const uint32_t *sk = reinterpret_cast<const uint32_t *>(tbuf);
+    const uint32_t *sv = reinterpret_cast<const uint32_t *>(tbuf + 64 * W);
+    const float2 *skm = reinterpret_cast<const float2 *>(tbuf + 128 * W);
+    const float2 *svm = reinterpret_cast<const float2 *>(tbuf + 128 * W + 128);
+    const int t0 = tile * 16;
+
+    // ---- logits: S^T = Q C^T per 8-token group
+    float lg[2][2];
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp) {
+      uint32_t kr[KB][2];
+      unpack_row<L>(sk + (grp * 8 + r) * W, c, kr);
+      float s[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb) mma_16816(s, qa[kb][0], 0u, qa[kb][1], 0u, kr[kb][0], kr[kb][1]);
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int tt = grp * 8 + 2 * c + e;
+        const float2 mm = skm[tt];
+        const float v = __fmaf_rn(s[e], mm.y * kscale, mm.x * qsc);
+        lg[grp][e] = (t0 + tt < n) ? v : -INFINITY;
+      }
+    }
+    // ---- online softmax (log2 domain), query r per lane quad
+    float mx = fmaxf(fmaxf(lg[0][0], lg[0][1]), fmaxf(lg[1][0], lg[1][1]));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+    const float m_new = fmaxf(m_run, mx);
+    if (__any_sync(0xffffffffu, m_new > m_run)) {
+      const float alpha = (m_new > m_run) ? ex2_approx(m_run - m_new) : 1.0f;   // m_run=-inf -> 0
+      l_run *= alpha;
+      mt_run *= alpha;
+      const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * c);       // query 2c
+      const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * c + 4);   // query 2c+1
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb) {
+        oacc[kb][0] *= a0;
+        oacc[kb][1] *= a1;
+        oacc[kb][2] *= a0;
+        oacc[kb][3] *= a1;
+      }
+      m_run = m_new;
+    }
+    float pw[2][2];
+#pragma unroll
+    for (int grp = 0; grp < 2; ++grp)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int tt = grp * 8 + 2 * c + e;
+        const bool ok = t0 + tt < n;
+        const float pr = ok ? ex2_approx(lg[grp][e] - m_run) : 0.0f;
+        const float2 vmm = svm[tt];
+        l_run += pr;
+        mt_run += ok ? pr * vmm.x : 0.0f;
+        pw[grp][e] = ok ? pr * (vmm.y * kappa) : 0.0f;
+      }
+    const uint32_t b0 = pack_half2(pw[0][0], pw[0][1]);
+    const uint32_t b1 = pack_half2(pw[1][0], pw[1][1]);
+
+    // ---- values: O^T += C^T P' (codes transposed in registers)
+    uint32_t vr0[KB][2], vr1[KB][2];
+    unpack_row<L>(sv + r * W, c, vr0);
+    unpack_row<L>(sv + (8 + r) * W, c, vr1);
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb) {
+      const uint32_t a0 = movmatrix_t(vr0[kb][0]);
+      const uint32_t a1 = movmatrix_t(vr0[kb][1]);
+      const uint32_t a2 = movmatrix_t(vr1[kb][0]);
+      const uint32_t a3 = movmatrix_t(vr1[kb][1]);
+      mma_16816(oacc[kb], a0, a1, a2, a3, b0, b1);
+    }
+    __syncwarp();
+    slotix = (slotix + 1) % DEC_NST;
+  }
+  cp_async_wait<0>();
+
+  // ---- quad totals of l and the min term (query r)
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  mt_run += __shfl_xor_sync(0xffffffffu, mt_run, 1);
+  mt_run += __shfl_xor_sync(0xffffffffu, mt_run, 2);
+
+  // ---- merge the 4 warps in shared memory (reuses the ring)
+  __syncthreads();
+  float *wo = reinterpret_cast<float *>(smem);                        // [warps][GMAX][128]
+  float *wst = wo + DEC_WARPS * DEC_GMAX * kD;                        // [warps][GMAX][3]
+  if (c == 0 && r < G) {
+    wst[(warp * DEC_GMAX + r) * 3 + 0] = m_run;
+    wst[(warp * DEC_GMAX + r) * 3 + 1] = l_run;
+    wst[(warp * DEC_GMAX + r) * 3 + 2] = mt_run;
+  }
+  constexpr float unscale = 16777216.0f / kappa;
+#pragma unroll
+  for (int kb = 0; kb < KB; ++kb) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      // slot r (hh=0) or 8+r (hh=1) of block kb belongs to lane group r/2, position (r%2) + 2hh
+      const int d = slot_dim<L>(r >> 1, 4 * kb + 2 * hh + (r & 1));
+      if (d >= 0) {
+        if (2 * c < G) wo[(warp * DEC_GMAX + 2 * c) * kD + d] = oacc[kb][2 * hh] * unscale;
+        if (2 * c + 1 < G) wo[(warp * DEC_GMAX + 2 * c + 1) * kD + d] = oacc[kb][2 * hh + 1] * unscale;
+      }
+    }
+  }
+  __syncthreads();
+  float *dst = p.part + ((int64_t)slab * p.NU + p.unit0 + split) * G * PART_STRIDE;
+  for (int i = threadIdx.x; i < G * kD; i += DEC_WARPS * 32) {
+    const int qh = i / kD, d = i % kD;
+    float M = -INFINITY;
+#pragma unroll
+    for (int wi = 0; wi < DEC_WARPS; ++wi) M = fmaxf(M, wst[(wi * DEC_GMAX + qh) * 3]);
+    float o = 0.0f, lsum = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int wi = 0; wi < DEC_WARPS; ++wi) {
+        const float mw = wst[(wi * DEC_GMAX + qh) * 3];
+        if (mw == -INFINITY) continue;
+        const float a = ex2_approx(mw - M);
+        o += a * (wo[(wi * DEC_GMAX + qh) * kD + d] + wst[(wi * DEC_GMAX + qh) * 3 + 2]);
+        lsum += a * wst[(wi * DEC_GMAX + qh) * 3 + 1];
+      }
+    }
+    dst[qh * PART_STRIDE + 4 + d] = o;
+    if (d == 0) {
+      dst[qh * PART_STRIDE + 0] = M;
+      dst[qh * PART_STRIDE + 1] = lsum;
+    }
+  }
+}
+
+// ---- FP16 block: one CTA of 128 threads per (sequence, layer, KV head)
+struct BufParams {
+  const uint16_t *bk, *bv;     // [B][Lyr][H][block][D]
+  int block, buf_len;
+  int B, Lyr, H, H_q, G, layer0, nL;
+  const uint16_t *q;
+  float c2;
+  float *part;
+  int NU, unit;
+};
+
+__global__ void __launch_bounds__(128) decode_buffer_kernel(const BufParams p) {
+  __shared__ float qs[DEC_GMAX][kD];
+  __shared__ float sc[DEC_GMAX][128];
+  __shared__ float red[DEC_GMAX][2];
+  const int slab = blockIdx.x;
+  const int h = slab % p.H, li = (slab / p.H) % p.nL, b = slab / (p.H * p.nL);
+  const int64_t pslab = ((int64_t)b * p.Lyr + p.layer0 + li) * p.H + h;
+  const int G = p.G, n = p.buf_len, tid = threadIdx.x;
+  for (int i = tid; i < G * kD; i += 128)
+    qs[i / kD][i % kD] = __half2float(__ushort_as_half(
+        p.q[(((int64_t)b * p.nL + li) * p.H_q + h * G + i / kD) * kD + i % kD]));
+  __syncthreads();
+  const uint16_t *kb = p.bk + pslab * p.block * kD;
+  const uint16_t *vb = p.bv + pslab * p.block * kD;
+  if (tid < n) {
+    for (int qh = 0; qh < G; ++qh) {
+      float acc = 0.0f;
+      for (int d = 0; d < kD; ++d) acc = fmaf(qs[qh][d], __half2float(__ushort_as_half(kb[(int64_t)tid * kD + d])), acc);
+      sc[qh][tid] = acc * p.c2;
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    for (int qh = 0; qh < G; ++qh) {
+      float mx = -INFINITY;
+      for (int t = tid; t < n; t += 32) mx = fmaxf(mx, sc[qh][t]);
+      for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      float s = 0.0f;
+      for (int t = tid; t < n; t += 32) s += ex2_approx(sc[qh][t] - mx);
+      for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      if (tid == 0) {
+        red[qh][0] = mx;
+        red[qh][1] = s;
+      }
+    }
+  }
+  __syncthreads();
+  float *dst = p.part + ((int64_t)slab * p.NU + p.unit) * G * PART_STRIDE;
+  for (int qh = 0; qh < G; ++qh) {
+    const float mx = red[qh][0];
+    float o = 0.0f;
+    if (n > 0)
+      for (int t = 0; t < n; ++t)
+        o = fmaf(ex2_approx(sc[qh][t] - mx), __half2float(__ushort_as_half(vb[(int64_t)t * kD + tid])), o);
+    dst[qh * PART_STRIDE + 4 + tid] = o;
+    if (tid == 0) {
+      dst[qh * PART_STRIDE + 0] = n > 0 ? mx : -INFINITY;
+      dst[qh * PART_STRIDE + 1] = n > 0 ? red[qh][1] : 0.0f;
+    }
+  }
+}
+
+// ---- merge all partials of a (sequence, layer, KV head): thread = head dim
+__global__ void __launch_bounds__(128) decode_merge_kernel(const float *__restrict__ part, int NU,
+                                                           int G, int H, int nL, int H_q,
+                                                           uint16_t *__restrict__ out) {
+  const int slab = blockIdx.x, d = threadIdx.x;
+  const int h = slab % H, li = (slab / H) % nL, b = slab / (H * nL);
+  for (int qh = 0; qh < G; ++qh) {
+    float M = -INFINITY;
+    for (int u = 0; u < NU; ++u) M = fmaxf(M, part[((int64_t)slab * NU + u) * G * PART_STRIDE + qh * PART_STRIDE]);
+    float o = 0.0f, l = 0.0f;
+    if (M != -INFINITY) {
+      for (int u = 0; u < NU; ++u) {
+        const float *pp = part + ((int64_t)slab * NU + u) * G * PART_STRIDE + qh * PART_STRIDE;
+        if (pp[0] == -INFINITY) continue;
+        const float a = ex2_approx(pp[0] - M);
+        o += a * pp[4 + d];
+        l += a * pp[1];
+      }
+    }
+    const float res = l > 0.0f ? o / l : 0.0f;
+    out[(((int64_t)b * nL + li) * H_q + h * G + qh) * kD + d] = __half_as_ushort(__float2half_rn(res));
+  }
+}
+
+// ---------------------------------------------------------------- host side
+template <int L>
+static int pool_smem_bytes(int G) {
+  return kQOff<L> + G * kD * 4;
+}
+
+template <int L>
+static cudaError_t launch_pool(const DecParams &p, int grid, cudaStream_t st) {
+  const int smem = pool_smem_bytes<L>(p.G);
+  static int attr_set = 0;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_pool_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         pool_smem_bytes<L>(DEC_GMAX));
+    if (e != cudaSuccess) return e;
+    attr_set = 1;
+  }
+  decode_pool_kernel<L><<<grid, DEC_WARPS * 32, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_pool_rt(int L, const DecParams &p, int grid, cudaStream_t st) {
+  switch (L) {
+    case 2: return launch_pool<2>(p, grid, st);
+    case 3: return launch_pool<3>(p, grid, st);
+    case 4: return launch_pool<4>(p, grid, st);
+    case 5: return launch_pool<5>(p, grid, st);
+    case 6: return launch_pool<6>(p, grid, st);
+    case 7: return launch_pool<7>(p, grid, st);
+    case 8: return launch_pool<8>(p, grid, st);
+    case 9: return launch_pool<9>(p, grid, st);
+    case 10: return launch_pool<10>(p, grid, st);
+    case 11: return launch_pool<11>(p, grid, st);
+    case 12: return launch_pool<12>(p, grid, st);
+    case 13: return launch_pool<13>(p, grid, st);
+    case 14: return launch_pool<14>(p, grid, st);
+    case 15: return launch_pool<15>(p, grid, st);
+    case 16: return launch_pool<16>(p, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// splits per slab for a pool of capacity cap (host knows only capacities)
+static int pool_splits(const semkv_cache &c, int n_layers, int cap) {
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t slabs = (int64_t)c.B * n_layers * c.H;
+  const int64_t target = (int64_t)sms * 12;           // ~4 waves of 3 CTAs per SM
+  int64_t S = (target + slabs - 1) / slabs;
+  const int64_t max_by_tiles = (cap / 16 + 15) / 16;  // keep >= 16 tiles (4 per warp) per unit
+  if (S > max_by_tiles) S = max_by_tiles;
+  if (S < 1) S = 1;
+  if (S > 64) S = 64;
+  return (int)S;
+}
+
+size_t decode_ws_bytes(const semkv_cache &c, int n_layers) {
+  const int Sh = pool_splits(c, n_layers, c.cap_high), Sl = pool_splits(c, n_layers, c.cap_low);
+  const int64_t slabs = (int64_t)c.B * n_layers * c.H;
+  const int G = c.H_q / c.H;
+  return (size_t)(slabs * (Sh + Sl + 1) * G * PART_STRIDE * sizeof(float));
+}
+
+cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, const uint16_t *q,
+                          uint16_t *out, float sm_scale, void *ws, cudaStream_t st) {
+  const int Sh = pool_splits(c, n_layers, c.cap_high), Sl = pool_splits(c, n_layers, c.cap_low);
+  const int NU = Sh + Sl + 1;
+  const int slabs = c.B * n_layers * c.H;
+  const int G = c.H_q / c.H;
+  DecParams p;
+  p.B = c.B;
+  p.Lyr = c.n_layers;
+  p.H = c.H;
+  p.H_q = c.H_q;
+  p.G = G;
+  p.layer0 = layer0;
+  p.nL = n_layers;
+  p.q = q;
+  p.c2 = sm_scale * kLog2eF;
+  p.part = reinterpret_cast<float *>(ws);
+  p.NU = NU;
+  cudaError_t e;
+  // high pool
+  p.kw = c.k_high; p.vw = c.v_high;
+  p.km = reinterpret_cast<const float2 *>(c.k_high_meta);
+  p.vm = reinterpret_cast<const float2 *>(c.v_high_meta);
+  p.count = c.n_high; p.cap = c.cap_high; p.unit0 = 0; p.S = Sh;
+  e = launch_pool_rt(c.L_high, p, slabs * Sh, st);
+  if (e != cudaSuccess) return e;
+  // low pool
+  p.kw = c.k_low; p.vw = c.v_low;
+  p.km = reinterpret_cast<const float2 *>(c.k_low_meta);
+  p.vm = reinterpret_cast<const float2 *>(c.v_low_meta);
+  p.count = c.n_low; p.cap = c.cap_low; p.unit0 = Sh; p.S = Sl;
+  e = launch_pool_rt(c.L_low, p, slabs * Sl, st);
+  if (e != cudaSuccess) return e;
+  // FP16 block
+  BufParams bp;
+  bp.bk = c.buf_k; bp.bv = c.buf_v; bp.block = c.block; bp.buf_len = c.buf_len;
+  bp.B = c.B; bp.Lyr = c.n_layers; bp.H = c.H; bp.H_q = c.H_q; bp.G = G;
+  bp.layer0 = layer0; bp.nL = n_layers; bp.q = q; bp.c2 = p.c2;
+  bp.part = p.part; bp.NU = NU; bp.unit = Sh + Sl;
+  decode_buffer_kernel<<<slabs, 128, 0, st>>>(bp);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_merge_kernel<<<slabs, 128, 0, st>>>(p.part, NU, G, c.H, n_layers, c.H_q, out);
+  return cudaGetLastError();
+}
+
+}  // namespace semkv

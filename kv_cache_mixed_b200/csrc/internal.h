@@ -1,0 +1,56 @@
+// internal.h -- host-side launchers shared by the C-ABI layer (not exported).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/semkv.h"
+
+namespace semkv {
+
+// Slot of each token within its class, and the high count per sequence.
+//   slot int32 [B][T_max], cnt_high int32 [B].
+cudaError_t launch_slot_scan(const uint8_t *mask, int64_t mask_bstride, const int32_t *seq_len,
+                             int len_const, int B, int T_max, int32_t *slot, int32_t *cnt_high,
+                             uint32_t *status, cudaStream_t st);
+
+struct QuantLaunch {
+  const uint16_t *k, *v;            // [B][Lyr][H][T_stride][128]
+  int B, Lyr, H, T_stride;
+  const int32_t *seq_len;           // NULL -> len_const
+  int len_const;
+  const uint8_t *mask;
+  int64_t mask_bstride;
+  const int32_t *slot;              // [B][T_stride]
+  const int32_t *cnt_high;          // [B]
+  int32_t *n_high, *n_low;          // device counts (bases before, advanced after)
+  uint32_t *k_high, *v_high, *k_low, *v_low;
+  float *k_high_meta, *v_high_meta, *k_low_meta, *v_low_meta;
+  int cap_high, cap_low, L_high, L_low;
+  uint32_t *status;
+};
+cudaError_t launch_quantize(const QuantLaunch &q, cudaStream_t st);
+
+cudaError_t launch_select(const float *score, int64_t score_bstride, const int32_t *seq_len,
+                          int len_const, int B, int T_max, int r_ppm, uint8_t *mask,
+                          int64_t mask_bstride, uint32_t *status, cudaStream_t st);
+
+cudaError_t launch_score_key_l2(const uint16_t *k, int64_t k_bstride, const int32_t *seq_len,
+                                int B, int T_max, int H, float *score, uint32_t *status,
+                                cudaStream_t st);
+
+size_t attn_mass_ws_bytes(int B, int T_max, int H, int H_q, int w);
+cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const uint16_t *q_win,
+                                   const int32_t *seq_len, int B, int T_max, int H, int H_q,
+                                   int w, float *score, void *ws, uint32_t *status,
+                                   cudaStream_t st);
+
+cudaError_t launch_buffer_append(const semkv_cache &c, const uint16_t *k_new,
+                                 const uint16_t *v_new, const float *score_new, int n_total,
+                                 int i0, int take, cudaStream_t st);
+
+size_t decode_ws_bytes(const semkv_cache &c, int n_layers);
+cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, const uint16_t *q,
+                          uint16_t *out, float sm_scale, void *ws, cudaStream_t st);
+
+}  // namespace semkv

@@ -183,6 +183,10 @@ def quantize_rows(xh: np.ndarray, L: int):
     """
     if xh.dtype != np.float16:
         raise ValueError("rows must be float16")
+    if xh.shape[0] == 0:
+        shp = xh.shape[:-1]
+        return (np.zeros(xh.shape, np.uint8), np.zeros(shp, np.float32), np.zeros(shp, np.float32),
+                np.zeros(shp, bool))
     x = xh.astype(np.float32)
     bad = ~np.all(np.isfinite(x), axis=-1)
     with np.errstate(invalid="ignore", divide="ignore", over="ignore"):
