@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--case", default=None, choices=["score", "select", "quantize", "decode"],
+                    help="profiling case: run only this stage, on the prefill workload cut to --layers layers")
+    ap.add_argument("--layers", type=int, default=4)
     return ap.parse_args()
 
 
@@ -374,8 +377,50 @@ def run_reference(args, rank):
             "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_case(args):
+    """One stage alone, repeated warmup+steps times, on the prefill workload cut
+    to args.layers layers (for ncu captures of a single kernel on a small case)."""
+    import torch
+
+    import kv_cache_mixed_b200 as kv
+    from inputs import synth
+    dev = torch.device("cuda")
+    wl = synth.scaled(synth.LLAMA_PREFILL, Lyr=args.layers)
+    B, Lyr, H, H_q, T, w = wl.B, wl.Lyr, wl.H, wl.H_q, wl.T, wl.w
+    k, v = synth.kv(wl, 0, dev)
+    q_win = synth.q_window(wl, 0, dev)
+    qdec = synth.decode_query(wl, 0, dev)
+    seq_len = synth.seq_lens(wl, 0).to(dev)
+    score = torch.empty((B, T), device=dev)
+    mask = torch.empty((B, T), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(qdec)
+    nh = kv.semkv_num_high(T, wl.r_ppm)
+    cache = kv.MixedCache(B, Lyr, H, H_q, wl.L_high, wl.L_low, wl.r_ppm, nh + 128, T - nh + 128)
+    kv.semkv_score(kv.SCORE_ATTN_MASS, k[:, Lyr - 1], k.stride(0), q_win, seq_len, B, T, H, H_q, w, score)
+    kv.semkv_select(score, seq_len, wl.r_ppm, mask)
+    kv.semkv_quantize(cache, k, v, seq_len, mask)
+    torch.cuda.synchronize()
+    for _ in range(args.warmup + args.steps):
+        if args.case == "score":
+            kv.semkv_score(kv.SCORE_ATTN_MASS, k[:, Lyr - 1], k.stride(0), q_win, seq_len, B, T, H, H_q, w, score)
+        elif args.case == "select":
+            kv.semkv_select(score, seq_len, wl.r_ppm, mask)
+        elif args.case == "quantize":
+            cache.n_high.zero_()
+            cache.n_low.zero_()
+            kv.semkv_quantize(cache, k, v, seq_len, mask)
+        else:
+            kv.semkv_decode_attn(cache, 0, Lyr, qdec, out)
+    torch.cuda.synchronize()
+    assert cache.status_flags() == 0
+    print(json.dumps({"case": args.case, "layers": Lyr, "ok": True}))
+
+
 def main():
     args = parse()
+    if args.case:
+        run_case(args)
+        return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     dist = None
