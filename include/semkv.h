@@ -51,6 +51,7 @@ typedef enum semkv_status {
 #define SEMKV_FLAG_NONFINITE 0x1u  /* a quantized row or a score held NaN/Inf; that row's output is unspecified */
 #define SEMKV_FLAG_CAPACITY  0x2u  /* a row did not fit its pool; it was not written                           */
 #define SEMKV_FLAG_SEQLEN    0x4u  /* seq_len[b] outside [0, T_max]; the sequence was skipped                  */
+#define SEMKV_FLAG_TIMEOUT   0x8u  /* a bounded wait for an asynchronous copy gave up; that output is unspecified */
 
 typedef enum semkv_score_kind {
   SEMKV_SCORE_ATTN_MASS = 0,   /* attention mass from the last w query rows (Table 1 "Attn."; Fig. 10) */
@@ -208,7 +209,7 @@ size_t semkv_decode_workspace_size(const semkv_cache *c, int32_t n_layers);
  */
 semkv_status semkv_decode_attn(const semkv_cache *c, int32_t layer0, int32_t n_layers,
                                const uint16_t *q, uint16_t *out, float sm_scale, void *ws,
-                               size_t ws_bytes, void *stream);
+                               size_t ws_bytes, uint32_t *status, void *stream);
 
 #ifdef __cplusplus
 }

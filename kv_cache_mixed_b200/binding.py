@@ -22,7 +22,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 SEMKV_OK = 0
 STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_WORKSPACE",
                 4: "ERR_CAPACITY", 5: "ERR_CUDA"}
-FLAG_NONFINITE, FLAG_CAPACITY, FLAG_SEQLEN = 0x1, 0x2, 0x4
+FLAG_NONFINITE, FLAG_CAPACITY, FLAG_SEQLEN, FLAG_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 SCORE_ATTN_MASS, SCORE_KEY_L2 = 0, 1
 FLUSH = 0x1
 
@@ -61,7 +61,8 @@ _lib_append_ws = _sig("semkv_append_workspace_size", _sz, [ctypes.POINTER(SemkvC
 _lib_append = _sig("semkv_append_block", _i32, [ctypes.POINTER(SemkvCache), _p, _p, _p, _i32, _u32, _p, _sz,
                                                 _p, _p])
 _lib_decode_ws = _sig("semkv_decode_workspace_size", _sz, [ctypes.POINTER(SemkvCache), _i32])
-_lib_decode = _sig("semkv_decode_attn", _i32, [ctypes.POINTER(SemkvCache), _i32, _i32, _p, _p, _f32, _p, _sz, _p])
+_lib_decode = _sig("semkv_decode_attn", _i32, [ctypes.POINTER(SemkvCache), _i32, _i32, _p, _p, _f32, _p, _sz, _p,
+                                                _p])
 
 EXPORTED = ["semkv_num_high", "semkv_digits_per_word", "semkv_words_per_row", "semkv_version",
             "semkv_score_workspace_size", "semkv_score", "semkv_select_workspace_size", "semkv_select",
@@ -213,5 +214,5 @@ def semkv_decode_attn(cache: MixedCache, layer0: int, n_layers: int, q: torch.Te
     """q, out fp16 [B][n_layers][H_q][128]."""
     ws = cache.workspace(("decode", n_layers), int(_lib_decode_ws(ctypes.byref(cache.c), n_layers)))
     _check(_lib_decode(ctypes.byref(cache.c), layer0, n_layers, _ptr(q), _ptr(out), sm_scale, _ptr(ws),
-                       ws.numel(), _stream(stream)), "semkv_decode_attn")
+                       ws.numel(), _ptr(cache.status), _stream(stream)), "semkv_decode_attn")
     return out

@@ -224,14 +224,14 @@ size_t semkv_decode_workspace_size(const semkv_cache *c, int32_t n_layers) {
 
 semkv_status semkv_decode_attn(const semkv_cache *c, int32_t layer0, int32_t n_layers,
                                const uint16_t *q, uint16_t *out, float sm_scale, void *ws,
-                               size_t ws_bytes, void *stream) {
+                               size_t ws_bytes, uint32_t *status, void *stream) {
   semkv_status s = check_cache(c);
   if (s != SEMKV_OK) return s;
   if (layer0 < 0 || n_layers <= 0 || layer0 + n_layers > c->n_layers) return SEMKV_ERR_INVALID_ARG;
   if (!al16(q) || !al16(out)) return SEMKV_ERR_INVALID_ARG;
   if (!(sm_scale > 0.0f) || sm_scale != sm_scale) return SEMKV_ERR_INVALID_ARG;
   if (!al16(ws) || ws_bytes < decode_ws_bytes(*c, n_layers)) return SEMKV_ERR_WORKSPACE;
-  return cuda_status(launch_decode(*c, layer0, n_layers, q, out, sm_scale, ws, S(stream)));
+  return cuda_status(launch_decode(*c, layer0, n_layers, q, out, sm_scale, ws, status, S(stream)));
 }
 
 }  // extern "C"

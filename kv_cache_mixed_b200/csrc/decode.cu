@@ -55,9 +55,10 @@ struct Geo {
   static_assert(split_part(L, 0) + split_part(L, 1) + split_part(L, 2) == N, "split must cover the word");
 };
 
-// digit j (0 = least significant) of word w into dig[j0 + j]
+// digit j (0 = least significant) of word w into dig[j0 + j].  Lr holds L at
+// run time so that every digit step stays one wide multiply.
 template <int L, int NDIG>
-__device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&dig)[NDIG], int j0) {
+__device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&dig)[NDIG], int j0, uint32_t Lr) {
   constexpr int NP = split_parts(L);
   uint32_t rest = w;
   int jb = j0;
@@ -77,9 +78,10 @@ __device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&dig)[NDIG], 
     uint32_t F = v * M;
 #pragma unroll
     for (int d = k - 1; d >= 0; --d) {
-      const unsigned long long t = (unsigned long long)F * (unsigned long long)L;
-      dig[jb + d] = (uint32_t)(t >> 32);
-      F = (uint32_t)t;
+      uint32_t lo, hi;
+      mul_wide(F, Lr, lo, hi);
+      dig[jb + d] = hi;
+      F = lo;
     }
     jb += k;
   }
@@ -89,23 +91,23 @@ __device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&dig)[NDIG], 
 // Its digit slot u = i*N + j (word i, digit j) sits in k-block u/4 at
 // position u%4; positions 0,1 are one f16x2 register, 2,3 the other.
 template <int L>
-__device__ __forceinline__ void unpack_row(const uint32_t *wrow, int c,
+__device__ __forceinline__ void unpack_row(const uint32_t *wrow, int c, uint32_t Lr,
                                            uint32_t (&reg)[Geo<L>::KB][2]) {
   using G = Geo<L>;
   constexpr int ND = G::KB * 4;
   uint32_t dig[ND];
+  // words past W of the row read the next bytes of the tile buffer: any 32-bit
+  // value unpacks to digits in [0, L) and those slots carry q = 0 (K) or are
+  // never written out (V), so no bounds check is needed
+  const uint32_t *wr = wrow + c * G::WPG;
 #pragma unroll
-  for (int i = 0; i < G::WPG; ++i) {
-    const int wi = c * G::WPG + i;
-    const uint32_t w = wi < G::W ? wrow[wi] : 0u;
-    extract_word<L, ND>(w, dig, i * G::N);
-  }
+  for (int i = 0; i < G::WPG; ++i) extract_word<L, ND>(wr[i], dig, i * G::N, Lr);
 #pragma unroll
   for (int u = G::WPG * G::N; u < ND; ++u) dig[u] = 0u;
 #pragma unroll
   for (int kb = 0; kb < G::KB; ++kb) {
-    reg[kb][0] = dig[4 * kb] | (dig[4 * kb + 1] << 16);
-    reg[kb][1] = dig[4 * kb + 2] | (dig[4 * kb + 3] << 16);
+    reg[kb][0] = __byte_perm(dig[4 * kb], dig[4 * kb + 1], 0x5410);
+    reg[kb][1] = __byte_perm(dig[4 * kb + 2], dig[4 * kb + 3], 0x5410);
   }
 }
 
@@ -130,12 +132,17 @@ struct DecParams {
   float c2;                         // sm_scale * log2(e)
   float *part;                      // [slabs][NU][G][PART_STRIDE]
   int NU, unit0, S;                 // units per slab, first unit of this launch, splits
+  uint32_t *status;
+  uint32_t Lrt;                     // the pool's level count (equals the template L)
 };
 
 constexpr int kMergeBytes = DEC_WARPS * DEC_GMAX * kD * 4 + DEC_WARPS * DEC_GMAX * 3 * 4;
 template <int L>
-constexpr int kQOff = (DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES > kMergeBytes)
-                          ? DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES : kMergeBytes;
+constexpr int kBarOff = (DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES > kMergeBytes)
+                            ? DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES : kMergeBytes;
+template <int L>
+constexpr int kQOff = kBarOff<L> + DEC_WARPS * DEC_NST * 8;
+constexpr int kWaitLimit = 1 << 20;         // mbarrier polls before a copy is declared lost
 
 template <int L>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
@@ -149,10 +156,17 @@ decode_pool_kernel(const DecParams p) {
   const int h = slab % p.H, li = (slab / p.H) % p.nL, b = slab / (p.H * p.nL);
   const int64_t pslab = ((int64_t)b * p.Lyr + p.layer0 + li) * p.H + h;
   const int G = p.G;
+  const uint32_t Lr = p.Lrt;                             // == L, opaque to the compiler
 
-  // ---- shared memory: per-warp tile rings, then the q rows
+  // ---- shared memory: per-warp tile rings, their mbarriers, then the q rows
   uint8_t *ring = smem + warp * DEC_NST * Gm::TILE_BYTES;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff<L>) + warp * DEC_NST;
   float *qs = reinterpret_cast<float *>(smem + kQOff<L>);   // [G][128]
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < DEC_NST; ++s) mbar_init(&bars[s], 1);
+    fence_mbar_init();
+  }
   for (int i = threadIdx.x; i < G * kD; i += DEC_WARPS * 32) {
     const int qh = i / kD, d = i % kD;
     const uint16_t hb = p.q[(((int64_t)b * p.nL + li) * p.H_q + h * G + qh) * kD + d];
@@ -191,27 +205,20 @@ decode_pool_kernel(const DecParams p) {
   const float2 *km = p.km + pslab * p.cap;
   const float2 *vm = p.vm + pslab * p.cap;
 
+  // one lane streams the warp's tiles: 4 bulk copies (K words, V words, K meta,
+  // V meta) completing on the slot's mbarrier
+  constexpr uint32_t kWB = 64 * W;                    // bytes of 16 rows of words
   auto issue = [&](int tile, int slotix) {
-    if (tile < te) {
+    if (lane == 0 && tile < te) {
       uint8_t *dst = ring + slotix * Gm::TILE_BYTES;
       const int t0 = tile * 16;
-      const uint8_t *kwb = reinterpret_cast<const uint8_t *>(kw + (int64_t)t0 * W);
-      const uint8_t *vwb = reinterpret_cast<const uint8_t *>(vw + (int64_t)t0 * W);
-      const uint8_t *kmb = reinterpret_cast<const uint8_t *>(km + t0);
-      const uint8_t *vmb = reinterpret_cast<const uint8_t *>(vm + t0);
-      constexpr int ch_w = 4 * W;           // 16-byte chunks of one 16-token word block
-      constexpr int total = 2 * ch_w + 16;
-      for (int i = lane; i < total; i += 32) {
-        const uint8_t *src;
-        int doff;
-        if (i < ch_w) { src = kwb + i * 16; doff = i * 16; }
-        else if (i < 2 * ch_w) { src = vwb + (i - ch_w) * 16; doff = i * 16; }
-        else if (i < 2 * ch_w + 8) { src = kmb + (i - 2 * ch_w) * 16; doff = i * 16; }
-        else { src = vmb + (i - 2 * ch_w - 8) * 16; doff = i * 16; }
-        cp_async16(dst + doff, src);
-      }
+      fence_proxy_async_smem();
+      mbar_expect_tx(&bars[slotix], 2 * kWB + 256);
+      bulk_g2s(dst, kw + (int64_t)t0 * W, kWB, &bars[slotix]);
+      bulk_g2s(dst + kWB, vw + (int64_t)t0 * W, kWB, &bars[slotix]);
+      bulk_g2s(dst + 2 * kWB, km + t0, 128, &bars[slotix]);
+      bulk_g2s(dst + 2 * kWB + 128, vm + t0, 128, &bars[slotix]);
     }
-    cp_async_commit();
   };
 
   float m_run = -INFINITY, l_run = 0.0f, mt_run = 0.0f;
@@ -227,11 +234,17 @@ decode_pool_kernel(const DecParams p) {
     next += DEC_WARPS;
   }
   int slotix = 0;
-  for (int tile = tb + warp; tile < te; tile += DEC_WARPS) {
+  uint32_t parity = 0;                 // bit s: parity of the next phase of slot s
+  bool lost = false;
+  int tile = tb + warp;
+  for (; tile < te; tile += DEC_WARPS) {
     issue(next, (slotix + DEC_NST - 1) % DEC_NST);
     next += DEC_WARPS;
-    cp_async_wait<DEC_NST - 1>();
-    __syncwarp();
+    if (!mbar_wait(&bars[slotix], (parity >> slotix) & 1u, kWaitLimit)) {
+      lost = true;
+      break;
+    }
+    parity ^= 1u << slotix;
     const uint8_t *tbuf = ring + slotix * Gm::TILE_BYTES;
     const uint32_t *sk = reinterpret_cast<const uint32_t *>(tbuf);
     const uint32_t *sv = reinterpret_cast<const uint32_t *>(tbuf + 64 * W);
@@ -244,7 +257,7 @@ decode_pool_kernel(const DecParams p) {
 #pragma unroll
     for (int grp = 0; grp < 2; ++grp) {
       uint32_t kr[KB][2];
-      unpack_row<L>(sk + (grp * 8 + r) * W, c, kr);
+      unpack_row<L>(sk + (grp * 8 + r) * W, c, Lr, kr);
       float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int kb = 0; kb < KB; ++kb) mma_16816(s, qa[kb][0], 0u, qa[kb][1], 0u, kr[kb][0], kr[kb][1]);
@@ -303,8 +316,8 @@ decode_pool_kernel(const DecParams p) {
 
     // ---- values: O^T += C^T P' (codes transposed in registers)
     uint32_t vr0[KB][2], vr1[KB][2];
-    unpack_row<L>(sv + r * W, c, vr0);
-    unpack_row<L>(sv + (8 + r) * W, c, vr1);
+    unpack_row<L>(sv + r * W, c, Lr, vr0);
+    unpack_row<L>(sv + (8 + r) * W, c, Lr, vr1);
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
       const uint32_t a0 = movmatrix_t(vr0[kb][0]);
@@ -317,7 +330,14 @@ decode_pool_kernel(const DecParams p) {
     __syncwarp();
     slotix = (slotix + 1) % DEC_NST;
   }
-  cp_async_wait<0>();
+  if (lost) {
+    // a copy did not arrive in time: flag it, and give the copies still in
+    // flight (tiles tile, tile+4, ... < next) a bounded chance to land before
+    // this CTA's shared memory is released
+    if (lane == 0) set_flag(p.status, SEMKV_FLAG_TIMEOUT);
+    for (int t2 = tile, s2 = slotix; t2 < next && t2 < te; t2 += DEC_WARPS, s2 = (s2 + 1) % DEC_NST)
+      mbar_wait(&bars[s2], (parity >> s2) & 1u, kWaitLimit);
+  }
 
   // ---- quad totals of l and the min term (query r)
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
@@ -524,7 +544,7 @@ size_t decode_ws_bytes(const semkv_cache &c, int n_layers) {
 }
 
 cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, const uint16_t *q,
-                          uint16_t *out, float sm_scale, void *ws, cudaStream_t st) {
+                          uint16_t *out, float sm_scale, void *ws, uint32_t *status, cudaStream_t st) {
   const int Sh = pool_splits(c, n_layers, c.cap_high), Sl = pool_splits(c, n_layers, c.cap_low);
   const int NU = Sh + Sl + 1;
   const int slabs = c.B * n_layers * c.H;
@@ -541,19 +561,20 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, const 
   p.c2 = sm_scale * kLog2eF;
   p.part = reinterpret_cast<float *>(ws);
   p.NU = NU;
+  p.status = status;
   cudaError_t e;
   // high pool
   p.kw = c.k_high; p.vw = c.v_high;
   p.km = reinterpret_cast<const float2 *>(c.k_high_meta);
   p.vm = reinterpret_cast<const float2 *>(c.v_high_meta);
-  p.count = c.n_high; p.cap = c.cap_high; p.unit0 = 0; p.S = Sh;
+  p.count = c.n_high; p.cap = c.cap_high; p.unit0 = 0; p.S = Sh; p.Lrt = (uint32_t)c.L_high;
   e = launch_pool_rt(c.L_high, p, slabs * Sh, st);
   if (e != cudaSuccess) return e;
   // low pool
   p.kw = c.k_low; p.vw = c.v_low;
   p.km = reinterpret_cast<const float2 *>(c.k_low_meta);
   p.vm = reinterpret_cast<const float2 *>(c.v_low_meta);
-  p.count = c.n_low; p.cap = c.cap_low; p.unit0 = Sh; p.S = Sl;
+  p.count = c.n_low; p.cap = c.cap_low; p.unit0 = Sh; p.S = Sl; p.Lrt = (uint32_t)c.L_low;
   e = launch_pool_rt(c.L_low, p, slabs * Sl, st);
   if (e != cudaSuccess) return e;
   // FP16 block

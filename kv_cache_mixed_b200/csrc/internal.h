@@ -51,6 +51,6 @@ cudaError_t launch_buffer_append(const semkv_cache &c, const uint16_t *k_new,
 
 size_t decode_ws_bytes(const semkv_cache &c, int n_layers);
 cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, const uint16_t *q,
-                          uint16_t *out, float sm_scale, void *ws, cudaStream_t st);
+                          uint16_t *out, float sm_scale, void *ws, uint32_t *status, cudaStream_t st);
 
 }  // namespace semkv

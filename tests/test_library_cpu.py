@@ -46,7 +46,7 @@ def test_invalid_arguments_rejected_before_launch(kv):
     INVALID, UNSUP, WS = 1, 2, 3
     # null cache
     assert b._lib_quant(None, None, None, 16, None, None, None, 0, None, None) == INVALID
-    assert b._lib_decode(None, 0, 1, None, None, 1.0, None, 0, None) == INVALID
+    assert b._lib_decode(None, 0, 1, None, None, 1.0, None, 0, None, None) == INVALID
     assert b._lib_append(None, None, None, None, 1, 0, None, 0, None, None) == INVALID
     # a cache with D != 128, bad levels, unaligned pointers, bad capacities
     def cache(**kw):
@@ -63,7 +63,7 @@ def test_invalid_arguments_rejected_before_launch(kv):
                      (dict(cap_high=17), INVALID), (dict(block=0), INVALID), (dict(buf_len=128), INVALID)]:
         c = cache(**kw)
         assert b._lib_decode(ctypes.byref(c), 0, 1, ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), 1.0,
-                             ctypes.c_void_p(0x10000), 1 << 20, None) == want, kw
+                             ctypes.c_void_p(0x10000), 1 << 20, None, None) == want, kw
     c = cache()
     c.k_low = 0x10008                              # misaligned pool
     assert b._lib_quant(ctypes.byref(c), ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), 16,
@@ -76,9 +76,9 @@ def test_invalid_arguments_rejected_before_launch(kv):
                         None, None) == WS
     # decode: layer range, bad scale
     assert b._lib_decode(ctypes.byref(c), 1, 1, ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), 1.0,
-                         ctypes.c_void_p(0x10000), 1 << 20, None) == INVALID
+                         ctypes.c_void_p(0x10000), 1 << 20, None, None) == INVALID
     assert b._lib_decode(ctypes.byref(c), 0, 1, ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), -1.0,
-                         ctypes.c_void_p(0x10000), 1 << 20, None) == INVALID
+                         ctypes.c_void_p(0x10000), 1 << 20, None, None) == INVALID
     # append: negative n, unknown flag
     assert b._lib_append(ctypes.byref(c), None, None, None, -1, 0, ctypes.c_void_p(0x10000), 1 << 20,
                          None, None) == INVALID
