@@ -142,6 +142,8 @@ constexpr int kBarOff = (DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES > kMergeBytes)
                             ? DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES : kMergeBytes;
 template <int L>
 constexpr int kQOff = kBarOff<L> + DEC_WARPS * DEC_NST * 8;
+static_assert(Geo<6>::TILE_BYTES % 16 == 0 && Geo<5>::TILE_BYTES % 16 == 0 && kMergeBytes % 16 == 0,
+              "tile buffers must keep 16-byte alignment for bulk copies");
 constexpr int kWaitLimit = 1 << 20;         // mbarrier polls before a copy is declared lost
 
 template <int L>
@@ -493,6 +495,9 @@ static cudaError_t launch_pool(const DecParams &p, int grid, cudaStream_t st) {
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(decode_pool_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          pool_smem_bytes<L>(DEC_GMAX));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(decode_pool_kernel<L>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     attr_set = 1;
   }
