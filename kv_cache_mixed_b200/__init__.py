@@ -2,7 +2,7 @@
 
 The kernels live in libsemkv.so (C ABI: include/semkv.h); this package is a
 thin binding with the same names.  Importing it fails loudly if the library
-has not been built (`python -m kv_cache_mixed_b200.build`).
+has not been built (`python kv_cache_mixed_b200/build.py`).
 """
 from .binding import (FLAG_CAPACITY, FLAG_NONFINITE, FLAG_SEQLEN, FLUSH, SCORE_ATTN_MASS,  # noqa: F401
                       SCORE_KEY_L2, EXPORTED, LIB_PATH, MixedCache, SemkvError, semkv_append_block,

@@ -16,7 +16,7 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libsemkv.so")
 
 if not os.path.exists(LIB_PATH):
-    raise ImportError(f"libsemkv.so not built at {LIB_PATH}; run `python -m kv_cache_mixed_b200.build`")
+    raise ImportError(f"libsemkv.so not built at {LIB_PATH}; run `python kv_cache_mixed_b200/build.py`")
 _lib = ctypes.CDLL(LIB_PATH)
 
 SEMKV_OK = 0

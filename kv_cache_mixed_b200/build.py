@@ -1,6 +1,8 @@
 """Build libsemkv.so (the CUDA kernels and the C ABI) for sm_100a, in-tree.
 
-    python -m kv_cache_mixed_b200.build        # or kv_cache_mixed_b200.build.build()
+    python kv_cache_mixed_b200/build.py [--force]
+
+(Run it as a file: importing the package loads the library this builds.)
 
 Objects go to kv_cache_mixed_b200/_build/, the library to
 kv_cache_mixed_b200/libsemkv.so.  A source newer than the library triggers a

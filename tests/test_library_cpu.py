@@ -14,8 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def kv():
-    from kv_cache_mixed_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__.build()
     import kv_cache_mixed_b200 as kv
     return kv
 
