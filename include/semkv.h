@@ -176,6 +176,33 @@ semkv_status semkv_quantize(semkv_cache *c, const uint16_t *k, const uint16_t *v
                             int32_t T_max, const int32_t *seq_len, const uint8_t *mask,
                             void *ws, size_t ws_bytes, uint32_t *status, void *stream);
 
+/*
+ * semkv_quantize without a caller workspace.  (The paper has no counterpart:
+ * this is a library convenience.)  For callers that cannot allocate device
+ * memory when they call in -- for example an inference engine that has handed
+ * all device memory to its own pool allocator, or a plugin host that forbids
+ * cudaMalloc on its hot path -- and so have no workspace to pass.  It computes
+ * exactly what semkv_quantize computes, with the workspace taken from a fixed
+ * array that the library keeps in device memory:
+ *   - the array holds SEMKV_NOALLOC_SCRATCH_BYTES on every GPU that loads the
+ *     library, until the process exits;
+ *   - sizes needing more (semkv_quantize_workspace_size(c->B, T_max) larger
+ *     than that, i.e. B*T_max above about one million tokens) are rejected
+ *     with SEMKV_ERR_WORKSPACE before anything is enqueued;
+ *   - the first call on a device looks up the array's device address on the
+ *     host (once per device, with that device current); make that first call
+ *     before any stream capture;
+ *   - every call on a device uses the same array, which keeps the last call's
+ *     contents: calls whose work overlaps on the GPU (other streams, other
+ *     threads) race, so serialize them;
+ *   - it calls no allocator: no cudaMalloc, cudaFree or allocating library.
+ * Arguments, results, flags and errors are otherwise those of semkv_quantize.
+ */
+#define SEMKV_NOALLOC_SCRATCH_BYTES (4u << 20)
+semkv_status semkv_quantize_noalloc(semkv_cache *c, const uint16_t *k, const uint16_t *v,
+                                    int32_t T_max, const int32_t *seq_len, const uint8_t *mask,
+                                    uint32_t *status, void *stream);
+
 /* ---- a5: generation-time block-exact path (Fig. 6) ------------------------- */
 
 size_t semkv_append_workspace_size(const semkv_cache *c);

@@ -57,6 +57,8 @@ _lib_select_ws = _sig("semkv_select_workspace_size", _sz, [_i32, _i32])
 _lib_select = _sig("semkv_select", _i32, [_p, _i64, _p, _i32, _i32, _i32, _i32, _p, _i64, _p, _sz, _p, _p])
 _lib_quant_ws = _sig("semkv_quantize_workspace_size", _sz, [_i32, _i32])
 _lib_quant = _sig("semkv_quantize", _i32, [ctypes.POINTER(SemkvCache), _p, _p, _i32, _p, _p, _p, _sz, _p, _p])
+_lib_quant_noalloc = _sig("semkv_quantize_noalloc", _i32, [ctypes.POINTER(SemkvCache), _p, _p, _i32, _p, _p, _p,
+                                                            _p])
 _lib_append_ws = _sig("semkv_append_workspace_size", _sz, [ctypes.POINTER(SemkvCache)])
 _lib_append = _sig("semkv_append_block", _i32, [ctypes.POINTER(SemkvCache), _p, _p, _p, _i32, _u32, _p, _sz,
                                                 _p, _p])
@@ -66,7 +68,8 @@ _lib_decode = _sig("semkv_decode_attn", _i32, [ctypes.POINTER(SemkvCache), _i32,
 
 EXPORTED = ["semkv_num_high", "semkv_digits_per_word", "semkv_words_per_row", "semkv_version",
             "semkv_score_workspace_size", "semkv_score", "semkv_select_workspace_size", "semkv_select",
-            "semkv_quantize_workspace_size", "semkv_quantize", "semkv_append_workspace_size",
+            "semkv_quantize_workspace_size", "semkv_quantize", "semkv_quantize_noalloc",
+            "semkv_append_workspace_size",
             "semkv_append_block", "semkv_decode_workspace_size", "semkv_decode_attn"]
 
 
@@ -200,6 +203,13 @@ def semkv_quantize(cache: MixedCache, k: torch.Tensor, v: torch.Tensor, seq_len:
     ws = cache.workspace("quant", int(_lib_quant_ws(cache.c.B, T_max)))
     _check(_lib_quant(ctypes.byref(cache.c), _ptr(k), _ptr(v), T_max, _ptr(seq_len), _ptr(mask), _ptr(ws),
                       ws.numel(), _ptr(cache.status), _stream(stream)), "semkv_quantize")
+
+
+def semkv_quantize_noalloc(cache: MixedCache, k: torch.Tensor, v: torch.Tensor, seq_len: torch.Tensor,
+                           mask: torch.Tensor, stream=None):
+    """semkv_quantize with the library's fixed scratch array instead of a workspace."""
+    _check(_lib_quant_noalloc(ctypes.byref(cache.c), _ptr(k), _ptr(v), k.shape[3], _ptr(seq_len), _ptr(mask),
+                              _ptr(cache.status), _stream(stream)), "semkv_quantize_noalloc")
 
 
 def semkv_append_block(cache: MixedCache, k_new, v_new, score_new, n: int, flags: int = 0, stream=None):
