@@ -55,6 +55,21 @@ def compare_pools(cache, k, v, masks, seq_len, L_high, L_low, layers=None, heads
                         assert np.array_equal(gm[:, 1].view(np.uint32), pool.scale.view(np.uint32)), (b, l, h)
 
 
+def check_mask_near_threshold(mask_gpu, score_ref, mask_ref, n_high):
+    """A GPU mask from the GPU's own (tolerance-level) scores may differ from the
+    oracle's mask only at tokens whose oracle score lies within the score
+    tolerance of the oracle's threshold score; it keeps exactly n_high ones."""
+    assert int(mask_gpu.sum()) == n_high
+    diff = np.nonzero(mask_gpu != mask_ref)[0]
+    if diff.size == 0:
+        return 0
+    order = np.lexsort((np.arange(score_ref.shape[0]), -score_ref))
+    thr = score_ref[order[n_high - 1]] if n_high > 0 else np.inf
+    band = SCORE_RTOL * abs(thr) * 2 + SCORE_ATOL * 2
+    assert np.all(np.abs(score_ref[diff] - thr) <= band), (diff, score_ref[diff], thr)
+    return int(diff.size)
+
+
 def check_attention(out_gpu, out_ref):
     o = out_gpu.astype(np.float64)
     rel = np.linalg.norm(o - out_ref) / max(np.linalg.norm(out_ref), 1e-30)
