@@ -33,6 +33,10 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
+# kernels one step launches: attention-mass score 4 (row stats, merge, column
+# sums, head sum), select 1, quantize 3 (slot scan, quantize+pack, count
+# advance), append 1, decode 4 (one pool kernel per level, FP16 block, merge)
+LAUNCHES_PER_STEP = 4 + 1 + 3 + 1 + 4
 METRIC = "KV quantize+pack GB/s (FP16 in) & mixed-prec decode-attn GB/s vs HBM roofline"
 KERNEL_SOURCES = ["kv_cache_mixed_b200/csrc/quantize.cu", "kv_cache_mixed_b200/csrc/common.cuh"]
 
@@ -247,7 +251,7 @@ def run_ours(args, rank, world, dist):
                      "bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 3), "traffic": traffic, "peak_source": peak_kind},
         "clocks": clk2.summary(),
-        "gpu_launches": 12 * args.steps,
+        "gpu_launches": LAUNCHES_PER_STEP * args.steps,
     }
     return res, (k, v, q_win, qdec, kn, vn, sn, seq_len, score, mask, out, cache, score_ws, fp16_in)
 

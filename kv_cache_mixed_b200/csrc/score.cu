@@ -8,14 +8,16 @@
 // attn_mass: the attention indicator (SemKV, Table 1 "Attn.", Fig. 10: its
 //   recomputation grows with T): s_j = sum over query heads and the last w
 //   window rows of softmax_j(q . k_j / sqrt(D)), causal.  Two passes over K on
-//   tensor cores (mma.sync m16n8k16, fp16 in, fp32 accumulate): pass 1 finds
-//   every row's max and sum of exponentials (online, split over T chunks,
-//   merged by a small kernel), pass 2 recomputes the logits and sums the
-//   normalised probabilities down each key column.  Column sums are reduced in
-//   a fixed order (warp shuffles, then warps, then KV heads), so the score is
-//   deterministic.
+//   tensor cores (fp16 in, fp32 accumulate): pass 1 finds every row's max and
+//   sum of exponentials (online, split over T chunks, merged by a small
+//   kernel), pass 2 recomputes the logits and sums the normalised
+//   probabilities down each key column.  Window groups of up to 256 rows per
+//   KV head run on tcgen05 with TMEM accumulators (attn_umma_kernel); wider
+//   groups on mma.sync m16n8k16.  Column sums are reduced in a fixed order, so
+//   the score is deterministic.
 #include "common.cuh"
 #include "internal.h"
+#include "umma.cuh"
 
 namespace semkv {
 
@@ -376,12 +378,260 @@ __global__ void __launch_bounds__(AM_WARPS * 32, 1) attn_colsum_kernel(const Att
   }
 }
 
+// ---- both passes on the 5th-generation tensor cores (tcgen05, TMEM accumulators)
+// CTA = (key chunk, KV head g, sequence b), 8 warps.  The Np <= 256 window rows
+// of g's query heads stay in shared memory; 128-key tiles stream through a
+// 4-deep cp.async ring, all in the 128-byte-swizzled K-major layout the MMA
+// descriptors describe.  Thread 0 issues the MMAs of tile i into one of two
+// TMEM accumulators while the warps run the epilogue of tile i-1.
+//   pass 1: D[rows][keys] = Q_g[rows] . K^T  (two M=128 halves of rows, N=128):
+//           each thread owns one row, keeps an online (max, sum of exp2) over
+//           its chunk, and writes one partial per (row, chunk);
+//   pass 2: D[keys][rows] = K . Q_g^T  (M=128 keys, N=Np): each thread owns one
+//           key (warps w and w+4 split the rows) and sums exp2(s*c1 - M'_r),
+//           M'_r = M_r + log2(Z_r); one partial per (head, key), summed over
+//           heads in order by attn_headsum_kernel.
+constexpr int UA_THREADS = 256;
+constexpr int UA_KEYS = 128;
+constexpr int UA_MAXN = 256;
+constexpr int UA_NST = 4;                         // key tiles in the ring
+constexpr int UA_QBYTES = UA_MAXN * 256;
+constexpr int UA_KBYTES = UA_KEYS * 256;
+constexpr int UA_OFF_Q = 0;
+constexpr int UA_OFF_K = UA_QBYTES;
+constexpr int UA_OFF_M = UA_OFF_K + UA_NST * UA_KBYTES;          // float [256] M'_r (pass 2)
+constexpr int UA_OFF_X = UA_OFF_M + UA_MAXN * 4;                  // float [2][128] half-sum exchange
+constexpr int UA_OFF_BAR = UA_OFF_X + 2 * 128 * 4;                // u64 [2]
+constexpr int UA_OFF_SLOT = UA_OFF_BAR + 16;
+constexpr int UA_SMEM = UA_OFF_SLOT + 16 + 1024;
+constexpr int kUmmaWait = 1 << 22;
+static_assert(UA_OFF_K % 1024 == 0 && UA_KBYTES % 1024 == 0, "operand blocks must be 1024-byte aligned");
+
+template <int PASS>
+__global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnParams p, int Np, int nchunk,
+                                                                   float *head_part) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quarter = warp & 3, half = warp >> 2;
+  const int len = p.seq_len[b];
+  if (len < 0 || len > p.T_max) return;            // flagged by the head-sum / merge kernels
+  const int ntile = (len + UA_KEYS - 1) / UA_KEYS;
+  const int tb = (int)((int64_t)ntile * chunk / nchunk), te = (int)((int64_t)ntile * (chunk + 1) / nchunk);
+
+  float *Ms = reinterpret_cast<float *>(smem + UA_OFF_M);
+  float *xch = reinterpret_cast<float *>(smem + UA_OFF_X);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + UA_OFF_BAR);
+  uint32_t *slot = reinterpret_cast<uint32_t *>(smem + UA_OFF_SLOT);
+  const uint32_t sbase = smem_u32(smem);
+  if (warp == 0) tmem_alloc(slot, 512);
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+  }
+  // resident window rows of head g (zero past Rg), and pass 2's row constants
+  {
+    const uint16_t *qg = p.q + ((int64_t)b * p.H_q + g * p.G) * p.w * kD;
+    for (int i = tid; i < Np * 16; i += UA_THREADS) {
+      const int r = i >> 4, c = i & 15;
+      const bool ok = r < p.Rg;
+      cp_async16_zfill(smem + UA_OFF_Q + sw128_offset(r, c, Np), qg + (ok ? (int64_t)r * kD + c * 8 : 0), ok);
+    }
+    if (PASS == 2) {
+      for (int r = tid; r < Np; r += UA_THREADS) {
+        float m = INFINITY;                          // rows that contribute nothing
+        if (r < p.Rg) {
+          const float2 st = p.stats[(int64_t)b * p.H_q * p.w + g * p.Rg + r];
+          if (st.y > 0.0f) m = st.x - __log2f(st.y);     // st.y = 1/Z
+        }
+        Ms[r] = m;
+      }
+    }
+    cp_async_commit();
+  }
+  const uint16_t *kg = p.k + (int64_t)b * p.kbs + (int64_t)g * p.T_max * kD;
+  auto stage_keys = [&](int tile) {
+    if (tile < te) {
+      uint8_t *kd = smem + UA_OFF_K + (tile % UA_NST) * UA_KBYTES;
+      const int t0 = tile * UA_KEYS;
+      for (int i = tid; i < UA_KEYS * 16; i += UA_THREADS) {
+        const int r = i >> 4, c = i & 15;
+        const bool ok = t0 + r < p.T_max;
+        cp_async16_zfill(kd + sw128_offset(r, c, UA_KEYS), kg + (ok ? (int64_t)(t0 + r) * kD + c * 8 : 0), ok);
+      }
+    }
+    cp_async_commit();
+  };
+  for (int i = 0; i < UA_NST - 2; ++i) stage_keys(tb + i);
+
+  __syncthreads();
+  const uint32_t tmem = *slot;
+  tc_fence_after();
+  const uint32_t qa = sbase + UA_OFF_Q;
+
+  auto issue_mma = [&](int tile) {        // thread 0 only
+    const uint32_t ka = sbase + UA_OFF_K + (tile % UA_NST) * UA_KBYTES;
+    const uint32_t acc = tmem + (tile & 1) * 256;
+    if (PASS == 1) {
+      const uint32_t idesc = umma_idesc_f16(128, UA_KEYS);
+      for (int hf = 0; hf * 128 < Np; ++hf) {
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t off = (ks & 3) * 32;
+          const uint64_t adesc = umma_desc_sw128(qa + (ks >> 2) * (Np * 128) + hf * 128 * 128 + off);
+          const uint64_t bdesc = umma_desc_sw128(ka + (ks >> 2) * (UA_KEYS * 128) + off);
+          umma_f16(acc + hf * 128, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+        }
+      }
+    } else {
+      const uint32_t idesc = umma_idesc_f16(UA_KEYS, Np);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint32_t off = (ks & 3) * 32;
+        const uint64_t adesc = umma_desc_sw128(ka + (ks >> 2) * (UA_KEYS * 128) + off);
+        const uint64_t bdesc = umma_desc_sw128(qa + (ks >> 2) * (Np * 128) + off);
+        umma_f16(acc, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+      }
+    }
+    umma_commit(&bars[tile & 1]);
+  };
+
+  // pass 1 state: this thread's row; pass 2: this thread's key and column half
+  const int row = half * 128 + quarter * 32 + lane;
+  const int pos = (PASS == 1 && row < p.Rg) ? len - p.w + row % p.w : -1;
+  float m_run = -INFINITY, l_run = 0.0f;
+  const int ncol_half = Np / 2;                    // pass 2: rows per warp half (Np is a multiple of 64)
+  bool lost = false;
+  int nwait = 0;                                   // completed phases, per accumulator
+
+  for (int tile = tb; tile <= te; ++tile) {
+    // issue tile `tile` (if any): its keys were staged two iterations ago
+    if (tile < te) {
+      stage_keys(tile + UA_NST - 2);               // slot of tile-2: its MMA was waited for last iteration
+      cp_async_wait<UA_NST - 2>();
+      fence_proxy_async_smem();
+      if (__syncthreads_or(lost)) break;           // an accumulator never arrived: stop issuing
+      if (tid == 0) {
+        tc_fence_after();
+        issue_mma(tile);
+      }
+    }
+    // epilogue of tile-1
+    const int et = tile - 1;
+    if (et >= tb) {
+      const int ab = et & 1;
+      if (mbar_wait(&bars[ab], (nwait >> ab) & 1, kUmmaWait)) nwait ^= 1 << ab;
+      else lost = true;
+      tc_fence_after();
+      const int t0 = et * UA_KEYS;
+      const bool edge = t0 + UA_KEYS - 1 > len - p.w;
+      if (PASS == 1) {
+        if (half * 128 < Np && !lost) {
+          const uint32_t la = tmem + ab * 256 + half * 128 + ((uint32_t)(quarter * 32) << 16);
+          float v[128];
+#pragma unroll
+          for (int cb = 0; cb < 4; ++cb) {
+            uint32_t u[32];
+            tmem_ld32(la + cb * 32, u);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float sv = __uint_as_float(u[j]) * p.c1;
+              v[cb * 32 + j] = (!edge || t0 + cb * 32 + j <= pos) ? sv : -INFINITY;
+            }
+          }
+          float mx = m_run;
+#pragma unroll
+          for (int j = 0; j < 128; j += 2) mx = fmax3_nan(mx, v[j], v[j + 1]);
+          if (mx != -INFINITY) {
+            float sum = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 128; ++j) sum += ex2_approx(v[j] - mx);
+            l_run = l_run * ex2_approx(m_run - mx) + sum;
+            m_run = mx;
+          }
+        }
+      } else {
+        const int key = t0 + quarter * 32 + lane;
+        const int c0 = half * ncol_half;
+        const uint32_t la = tmem + ab * 256 + c0 + ((uint32_t)(quarter * 32) << 16);
+        float acc = 0.0f;
+        for (int cb = 0; cb < (lost ? 0 : ncol_half); cb += 32) {
+          uint32_t u[32];
+          tmem_ld32(la + cb, u);
+          tmem_ld_wait();
+          const float4 *M4 = reinterpret_cast<const float4 *>(Ms + c0 + cb);
+          if (!edge) {
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 m4 = M4[j4];
+              acc += ex2_approx(__uint_as_float(u[4 * j4 + 0]) * p.c1 - m4.x);
+              acc += ex2_approx(__uint_as_float(u[4 * j4 + 1]) * p.c1 - m4.y);
+              acc += ex2_approx(__uint_as_float(u[4 * j4 + 2]) * p.c1 - m4.z);
+              acc += ex2_approx(__uint_as_float(u[4 * j4 + 3]) * p.c1 - m4.w);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int r = c0 + cb + j;
+              const bool vis = r < p.Rg && key <= len - p.w + r % p.w;
+              acc += vis ? ex2_approx(__uint_as_float(u[j]) * p.c1 - Ms[r]) : 0.0f;
+            }
+          }
+        }
+        // the two column halves of this key: warp w+4 hands its sum to warp w
+        float *xb = xch + ab * 128;                // by accumulator: the next write to it follows a barrier
+        if (half == 1) xb[quarter * 32 + lane] = acc;
+        tc_fence_before();
+        __syncthreads();
+        if (half == 0 && key < p.T_max)
+          head_part[((int64_t)b * p.H + g) * p.T_max + key] = key < len ? acc + xb[quarter * 32 + lane] : 0.0f;
+        continue;
+      }
+      tc_fence_before();
+    }
+  }
+  if (PASS == 1) {
+    if (half * 128 < Np && row < p.Rg) {
+      const int hrow = (g * p.G + row / p.w) * p.w + row % p.w;    // h*w + i
+      p.part[((int64_t)b * p.H_q * p.w + hrow) * p.nchunk + chunk] = make_float2(m_run, l_run);
+    }
+  }
+  cp_async_wait<0>();
+  if (__syncthreads_or(lost) && tid == 0) {
+    // drain: wait (bounded) for whatever MMAs are still in flight before TMEM is freed
+    set_flag(p.status, SEMKV_FLAG_TIMEOUT);
+    for (int ab = 0; ab < 2; ++ab) mbar_wait(&bars[ab], (nwait >> ab) & 1, kUmmaWait / 64);
+  }
+  __syncthreads();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// score[b][j] = sum over KV heads, in order, of the per-head column partials
+__global__ void attn_headsum_kernel(const AttnParams p, const float *__restrict__ head_part) {
+  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (int64_t)p.B * p.T_max) return;
+  const int b = (int)(idx / p.T_max), j = (int)(idx % p.T_max);
+  const int len = p.seq_len[b];
+  if (len < 0 || len > p.T_max) {
+    p.score[idx] = 0.0f;
+    if (j == 0) set_flag(p.status, SEMKV_FLAG_SEQLEN);
+    return;
+  }
+  float s = 0.0f;
+  if (j < len)
+    for (int g = 0; g < p.H; ++g) s += head_part[((int64_t)b * p.H + g) * p.T_max + j];
+  p.score[idx] = s;
+}
+
 size_t attn_mass_ws_bytes(int B, int T_max, int H, int H_q, int w) {
-  (void)H;
   const int64_t rows = (int64_t)B * H_q * w;
   const int ntile = (T_max + AM_TILE - 1) / AM_TILE;
   const int nchunk = ntile < 64 ? ntile : 64;
-  return (size_t)(rows * nchunk * sizeof(float2) + rows * sizeof(float2) + 256);
+  const size_t parts = (size_t)(rows * nchunk * sizeof(float2) + rows * sizeof(float2) + 256);
+  return (parts + 255) / 256 * 256 + (size_t)B * H * T_max * sizeof(float) + 256;
 }
 
 cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const uint16_t *q_win,
@@ -405,17 +655,44 @@ cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const u
   int dev = 0, sms = 0;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  int want = (2 * sms + H * p.nrb * B - 1) / (H * p.nrb * B);
-  p.nchunk = want < 1 ? 1 : (want > ntile ? ntile : (want > 64 ? 64 : want));
   p.c1 = kLog2e / sqrtf((float)kD);
   const int64_t rows = (int64_t)B * H_q * w;
   const int nchunk_ws = ntile < 64 ? ntile : 64;
   p.part = reinterpret_cast<float2 *>(ws);
   p.stats = reinterpret_cast<float2 *>(reinterpret_cast<char *>(ws) + rows * nchunk_ws * sizeof(float2));
+  const size_t parts = (size_t)(rows * nchunk_ws * sizeof(float2) + rows * sizeof(float2) + 256);
+  float *head_part = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) + (parts + 255) / 256 * 256);
   p.score = score;
   p.status = status;
+  cudaError_t e;
+  const int Np = (p.Rg + 63) / 64 * 64;       // two column halves of whole 32-column loads
+  if (Np <= UA_MAXN) {
+    // tcgen05 path: one CTA per SM (all of TMEM), about one wave of CTAs
+    const int utiles = (T_max + UA_KEYS - 1) / UA_KEYS;
+    int nch = sms / (H * B);                  // whole waves only
+    nch = nch < 1 ? 1 : (nch > utiles ? utiles : (nch > 64 ? 64 : nch));
+    p.nchunk = nch;
+    e = cudaFuncSetAttribute(attn_umma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, UA_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(attn_umma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, UA_SMEM);
+    if (e != cudaSuccess) return e;
+    attn_umma_kernel<1><<<dim3(nch, H, B), UA_THREADS, UA_SMEM, st>>>(p, Np, nch, head_part);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_merge_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_umma_kernel<2><<<dim3(nch, H, B), UA_THREADS, UA_SMEM, st>>>(p, Np, nch, head_part);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    attn_headsum_kernel<<<(unsigned)(((int64_t)B * T_max + 255) / 256), 256, 0, st>>>(p, head_part);
+    return cudaGetLastError();
+  }
+  // mma.sync path for window groups wider than 256 rows
+  int want = (2 * sms + H * p.nrb * B - 1) / (H * p.nrb * B);
+  p.nchunk = want < 1 ? 1 : (want > ntile ? ntile : (want > 64 ? 64 : want));
   attn_rowstats_kernel<<<dim3(p.nchunk, H * p.nrb, B), AM_WARPS * 32, 0, st>>>(p);
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_merge_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
   e = cudaGetLastError();

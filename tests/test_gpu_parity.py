@@ -264,7 +264,11 @@ def test_key_l2_bit_exact(kdist):
         assert not s[b, T:].any()
 
 
-@pytest.mark.parametrize("H,H_q,w,lens", [(2, 8, 64, [700, 50]), (8, 32, 64, [2048, 1500]), (1, 4, 16, [333, 5])])
+# window groups of 256 rows (the shipped shape), 64 and 129 (padded row tiles,
+# sequences shorter than the window) and 512 rows (wider than one tensor-memory
+# accumulator: the mma.sync path)
+@pytest.mark.parametrize("H,H_q,w,lens", [(2, 8, 64, [700, 50]), (8, 32, 64, [2048, 1500]), (1, 4, 16, [333, 5]),
+                                          (2, 6, 43, [517, 40]), (1, 8, 64, [1000, 64])])
 def test_attn_mass_within_tolerance(H, H_q, w, lens):
     kv = kv_mod()
     T = max(lens)
