@@ -45,14 +45,25 @@ __host__ __device__ constexpr int split_part(int L, int i) {
 }
 __host__ __device__ constexpr int split_parts(int L) { return (L == 7 || L == 11) ? 3 : 2; }
 
+// Pair path (L <= 6): one wide multiply by L^2 yields two digits at once,
+// hi = c_{j+1} * L + c_j, and a shared-memory table of L^2 entries turns hi
+// into the f16x2 operand (c_j, c_{j+1}).  Every part of these levels starts on
+// an even digit and only the top part can have odd length, so with the word
+// stride in slots rounded up to even (L = 5: 13 digits in 14 slots) every pair
+// stays inside one part; an odd top part leads with one single-digit step.
+__host__ __device__ constexpr bool use_pairs(int L) { return L <= 6; }
+
 template <int L>
 struct Geo {
   static constexpr int N = digits_per_word(L);       // digits per word
   static constexpr int W = words_per_row(L);         // words per row
+  static constexpr int S = use_pairs(L) ? N + (N & 1) : N;   // slots per word
   static constexpr int WPG = (W + 3) / 4;            // words per lane group (lane % 4)
-  static constexpr int KB = (WPG * N + 3) / 4;       // 16-slot k-blocks
+  static constexpr int KB = (WPG * S + 3) / 4;       // 16-slot k-blocks
   static constexpr int TILE_BYTES = 16 * W * 4 * 2 + 16 * 8 * 2;
   static_assert(split_part(L, 0) + split_part(L, 1) + split_part(L, 2) == N, "split must cover the word");
+  static_assert(!use_pairs(L) || (split_part(L, 0) % 2 == 0 && (split_parts(L) == 2 || split_part(L, 1) % 2 == 0)),
+                "pair path needs even parts below the top part");
 };
 
 // digit j (0 = least significant) of word w into dig[j0 + j].  Lr holds L at
@@ -87,27 +98,78 @@ __device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&dig)[NDIG], 
   }
 }
 
+// pair path: f16x2 registers of slot pairs (j0 + 2m, j0 + 2m + 1) into pr[j0/2 + m]
+template <int L, int NPR>
+__device__ __forceinline__ void extract_word_pairs(uint32_t w, uint32_t (&pr)[NPR], int j0, uint32_t Lr,
+                                                   uint32_t L2r, const uint32_t *lut) {
+  constexpr int NP = split_parts(L);
+  uint32_t rest = w;
+  int jb = j0;
+#pragma unroll
+  for (int pi = 0; pi < NP; ++pi) {
+    const int k = split_part(L, pi);
+    uint32_t v;
+    if (pi < NP - 1) {
+      const uint32_t P = (uint32_t)ipow(L, k);
+      const uint32_t qq = rest / P;
+      v = rest - qq * P;
+      rest = qq;
+    } else {
+      v = rest;
+    }
+    const uint32_t M = (uint32_t)(((1ull << 32) + ipow(L, k) - 1) / ipow(L, k));
+    uint32_t F = v * M;
+    if (k & 1) {                       // odd top part: its top digit alone, upper half zero
+      uint32_t lo, hi;
+      mul_wide(F, Lr, lo, hi);
+      pr[(jb + k - 1) >> 1] = hi;
+      F = lo;
+    }
+#pragma unroll
+    for (int m = k / 2 - 1; m >= 0; --m) {
+      uint32_t lo, hi;
+      mul_wide(F, L2r, lo, hi);
+      pr[(jb >> 1) + m] = lut[hi];
+      F = lo;
+    }
+    jb += k;
+  }
+}
+
 // The lane group c = lane % 4 owns words c*WPG .. c*WPG+WPG-1 of a token row.
-// Its digit slot u = i*N + j (word i, digit j) sits in k-block u/4 at
+// Its digit slot u = i*S + j (word i, digit j) sits in k-block u/4 at
 // position u%4; positions 0,1 are one f16x2 register, 2,3 the other.
 template <int L>
-__device__ __forceinline__ void unpack_row(const uint32_t *wrow, int c, uint32_t Lr,
-                                           uint32_t (&reg)[Geo<L>::KB][2]) {
+__device__ __forceinline__ void unpack_row(const uint32_t *wrow, int c, uint32_t Lr, uint32_t L2r,
+                                           const uint32_t *lut, uint32_t (&reg)[Geo<L>::KB][2]) {
   using G = Geo<L>;
   constexpr int ND = G::KB * 4;
-  uint32_t dig[ND];
   // words past W of the row read the next bytes of the tile buffer: any 32-bit
   // value unpacks to digits in [0, L) and those slots carry q = 0 (K) or are
   // never written out (V), so no bounds check is needed
   const uint32_t *wr = wrow + c * G::WPG;
+  if constexpr (use_pairs(L)) {
+    uint32_t pr[ND / 2];
 #pragma unroll
-  for (int i = 0; i < G::WPG; ++i) extract_word<L, ND>(wr[i], dig, i * G::N, Lr);
+    for (int i = 0; i < G::WPG; ++i) extract_word_pairs<L, ND / 2>(wr[i], pr, i * G::S, Lr, L2r, lut);
 #pragma unroll
-  for (int u = G::WPG * G::N; u < ND; ++u) dig[u] = 0u;
+    for (int u = (G::WPG * G::S) / 2; u < ND / 2; ++u) pr[u] = 0u;
 #pragma unroll
-  for (int kb = 0; kb < G::KB; ++kb) {
-    reg[kb][0] = __byte_perm(dig[4 * kb], dig[4 * kb + 1], 0x5410);
-    reg[kb][1] = __byte_perm(dig[4 * kb + 2], dig[4 * kb + 3], 0x5410);
+    for (int kb = 0; kb < G::KB; ++kb) {
+      reg[kb][0] = pr[2 * kb];
+      reg[kb][1] = pr[2 * kb + 1];
+    }
+  } else {
+    uint32_t dig[ND];
+#pragma unroll
+    for (int i = 0; i < G::WPG; ++i) extract_word<L, ND>(wr[i], dig, i * G::N, Lr);
+#pragma unroll
+    for (int u = G::WPG * G::N; u < ND; ++u) dig[u] = 0u;
+#pragma unroll
+    for (int kb = 0; kb < G::KB; ++kb) {
+      reg[kb][0] = __byte_perm(dig[4 * kb], dig[4 * kb + 1], 0x5410);
+      reg[kb][1] = __byte_perm(dig[4 * kb + 2], dig[4 * kb + 3], 0x5410);
+    }
   }
 }
 
@@ -115,9 +177,10 @@ __device__ __forceinline__ void unpack_row(const uint32_t *wrow, int c, uint32_t
 template <int L>
 __device__ __forceinline__ int slot_dim(int c, int u) {
   using G = Geo<L>;
-  const int wi = c * G::WPG + u / G::N;
-  const int d = wi * G::N + u % G::N;
-  return (u < G::WPG * G::N && wi < G::W && d < kD) ? d : -1;
+  const int wi = c * G::WPG + u / G::S;
+  const int j = u % G::S;
+  const int d = wi * G::N + j;
+  return (u < G::WPG * G::S && j < G::N && wi < G::W && d < kD) ? d : -1;
 }
 
 struct DecParams {
@@ -145,6 +208,7 @@ constexpr int kQOff = kBarOff<L> + DEC_WARPS * DEC_NST * 8;
 static_assert(Geo<6>::TILE_BYTES % 16 == 0 && Geo<5>::TILE_BYTES % 16 == 0 && kMergeBytes % 16 == 0,
               "tile buffers must keep 16-byte alignment for bulk copies");
 constexpr int kWaitLimit = 1 << 20;         // mbarrier polls before a copy is declared lost
+constexpr int kLutBytes = 64 * 4;           // pair table, L*L <= 36 entries
 
 template <int L>
 __global__ void __launch_bounds__(DEC_WARPS * 32)
@@ -159,16 +223,20 @@ decode_pool_kernel(const DecParams p) {
   const int64_t pslab = ((int64_t)b * p.Lyr + p.layer0 + li) * p.H + h;
   const int G = p.G;
   const uint32_t Lr = p.Lrt;                             // == L, opaque to the compiler
+  const uint32_t L2r = Lr * Lr;
 
   // ---- shared memory: per-warp tile rings, their mbarriers, then the q rows
   uint8_t *ring = smem + warp * DEC_NST * Gm::TILE_BYTES;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff<L>) + warp * DEC_NST;
-  float *qs = reinterpret_cast<float *>(smem + kQOff<L>);   // [G][128]
+  uint32_t *lut = reinterpret_cast<uint32_t *>(smem + kQOff<L>);      // [L*L] digit pairs (pair path)
+  float *qs = reinterpret_cast<float *>(smem + kQOff<L> + kLutBytes);  // [G][128]
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < DEC_NST; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
+  if (use_pairs(L))
+    for (int i = threadIdx.x; i < L * L; i += DEC_WARPS * 32) lut[i] = (uint32_t)(i % L) | ((uint32_t)(i / L) << 16);
   for (int i = threadIdx.x; i < G * kD; i += DEC_WARPS * 32) {
     const int qh = i / kD, d = i % kD;
     const uint16_t hb = p.q[(((int64_t)b * p.nL + li) * p.H_q + h * G + qh) * kD + d];
@@ -259,7 +327,7 @@ decode_pool_kernel(const DecParams p) {
 #pragma unroll
     for (int grp = 0; grp < 2; ++grp) {
       uint32_t kr[KB][2];
-      unpack_row<L>(sk + (grp * 8 + r) * W, c, Lr, kr);
+      unpack_row<L>(sk + (grp * 8 + r) * W, c, Lr, L2r, lut, kr);
       float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int kb = 0; kb < KB; ++kb) mma_16816(s, qa[kb][0], 0u, qa[kb][1], 0u, kr[kb][0], kr[kb][1]);
@@ -318,8 +386,8 @@ decode_pool_kernel(const DecParams p) {
 
     // ---- values: O^T += C^T P' (codes transposed in registers)
     uint32_t vr0[KB][2], vr1[KB][2];
-    unpack_row<L>(sv + r * W, c, Lr, vr0);
-    unpack_row<L>(sv + (8 + r) * W, c, Lr, vr1);
+    unpack_row<L>(sv + r * W, c, Lr, L2r, lut, vr0);
+    unpack_row<L>(sv + (8 + r) * W, c, Lr, L2r, lut, vr1);
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
       const uint32_t a0 = movmatrix_t(vr0[kb][0]);
@@ -485,7 +553,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float *__restri
 // ---------------------------------------------------------------- host side
 template <int L>
 static int pool_smem_bytes(int G) {
-  return kQOff<L> + G * kD * 4;
+  return kQOff<L> + kLutBytes + G * kD * 4;
 }
 
 template <int L>
