@@ -530,26 +530,25 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
       if (PASS == 1) {
         if (half * 128 < Np && !lost) {
           const uint32_t la = tmem + ab * 256 + half * 128 + ((uint32_t)(quarter * 32) << 16);
+          // raw logits of this row for the 128 keys (c1 > 0: the max commutes with the scaling)
           float v[128];
 #pragma unroll
-          for (int cb = 0; cb < 4; ++cb) {
-            uint32_t u[32];
-            tmem_ld32(la + cb * 32, u);
-            tmem_ld_wait();
+          for (int cb = 0; cb < 4; ++cb) tmem_ld32(la + cb * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[cb * 32]));
+          tmem_ld_wait();
+          if (edge) {
+            const int lim = pos - t0;                // keys t0 + j with j > lim are masked
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float sv = __uint_as_float(u[j]) * p.c1;
-              v[cb * 32 + j] = (!edge || t0 + cb * 32 + j <= pos) ? sv : -INFINITY;
-            }
+            for (int j = 0; j < 128; ++j) v[j] = j <= lim ? v[j] : -INFINITY;
           }
-          float mx = m_run;
+          float mr = v[0];
 #pragma unroll
-          for (int j = 0; j < 128; j += 2) mx = fmax3_nan(mx, v[j], v[j + 1]);
+          for (int j = 1; j < 127; j += 2) mr = fmax3_nan(mr, v[j], v[j + 1]);
+          const float mx = fmax_nan(m_run, fmax_nan(mr, v[127]) * p.c1);
           if (mx != -INFINITY) {
-            float sum = 0.0f;
+            float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-            for (int j = 0; j < 128; ++j) sum += ex2_approx(v[j] - mx);
-            l_run = l_run * ex2_approx(m_run - mx) + sum;
+            for (int j = 0; j < 128; ++j) sum[j & 3] += ex2_approx(__fmaf_rn(v[j], p.c1, -mx));
+            l_run = l_run * ex2_approx(m_run - mx) + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
             m_run = mx;
           }
         }
@@ -557,30 +556,35 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
         const int key = t0 + quarter * 32 + lane;
         const int c0 = half * ncol_half;
         const uint32_t la = tmem + ab * 256 + c0 + ((uint32_t)(quarter * 32) << 16);
-        float acc = 0.0f;
-        for (int cb = 0; cb < (lost ? 0 : ncol_half); cb += 32) {
-          uint32_t u[32];
-          tmem_ld32(la + cb, u);
+        float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int cb = 0; cb < (lost ? 0 : ncol_half); cb += 64) {
+          uint32_t u[64];
+          tmem_ld32(la + cb, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+          tmem_ld32(la + cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
           tmem_ld_wait();
-          const float4 *M4 = reinterpret_cast<const float4 *>(Ms + c0 + cb);
+          const int nc = ncol_half - cb < 64 ? 32 : 64;   // ncol_half is a multiple of 32
           if (!edge) {
+            const float4 *M4 = reinterpret_cast<const float4 *>(Ms + c0 + cb);
 #pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
+            for (int j4 = 0; j4 < 16; ++j4) {
+              if (j4 * 4 >= nc) break;
               const float4 m4 = M4[j4];
-              acc += ex2_approx(__uint_as_float(u[4 * j4 + 0]) * p.c1 - m4.x);
-              acc += ex2_approx(__uint_as_float(u[4 * j4 + 1]) * p.c1 - m4.y);
-              acc += ex2_approx(__uint_as_float(u[4 * j4 + 2]) * p.c1 - m4.z);
-              acc += ex2_approx(__uint_as_float(u[4 * j4 + 3]) * p.c1 - m4.w);
+              acc4[0] += ex2_approx(__fmaf_rn(__uint_as_float(u[4 * j4 + 0]), p.c1, -m4.x));
+              acc4[1] += ex2_approx(__fmaf_rn(__uint_as_float(u[4 * j4 + 1]), p.c1, -m4.y));
+              acc4[2] += ex2_approx(__fmaf_rn(__uint_as_float(u[4 * j4 + 2]), p.c1, -m4.z));
+              acc4[3] += ex2_approx(__fmaf_rn(__uint_as_float(u[4 * j4 + 3]), p.c1, -m4.w));
             }
           } else {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
+            for (int j = 0; j < 64; ++j) {
+              if (j >= nc) break;
               const int r = c0 + cb + j;
               const bool vis = r < p.Rg && key <= len - p.w + r % p.w;
-              acc += vis ? ex2_approx(__uint_as_float(u[j]) * p.c1 - Ms[r]) : 0.0f;
+              acc4[j & 3] += vis ? ex2_approx(__fmaf_rn(__uint_as_float(u[j]), p.c1, -Ms[r])) : 0.0f;
             }
           }
         }
+        const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
         // the two column halves of this key: warp w+4 hands its sum to warp w
         float *xb = xch + ab * 128;                // by accumulator: the next write to it follows a barrier
         if (half == 1) xb[quarter * 32 + lane] = acc;
