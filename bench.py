@@ -41,7 +41,7 @@ METRIC = "KV quantize+pack GB/s (FP16 in) & mixed-prec decode-attn GB/s vs HBM r
 KERNEL_SOURCES = ["kv_cache_mixed_b200/csrc/quantize.cu", "kv_cache_mixed_b200/csrc/common.cuh"]
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=10)
@@ -52,7 +52,41 @@ def parse():
     ap.add_argument("--case", default=None, choices=["score", "select", "quantize", "decode"],
                     help="profiling case: run only this stage, on the prefill workload cut to --layers layers")
     ap.add_argument("--layers", type=int, default=4)
-    return ap.parse_args()
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------------ ranks
+def init_ranks(backend="nccl", timeout_s=120):
+    """(rank, world, torch.distributed or None) from the torchrun environment.
+    Replicas only: the ranks exchange nothing on the data path, just a barrier
+    around the timed region and a max-reduction of the step time."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if world <= 1:
+        return rank, world, None
+    import datetime
+
+    import torch
+    import torch.distributed as tdist
+    if backend == "nccl":
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
+    tdist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return rank, world, tdist
+
+
+def max_over_ranks(ms, dist, device):
+    """The slowest rank's time (every rank takes this collective, in the same order)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(world, bytes_per_rank, ms):
+    """Whole-job GB/s: the bytes every rank processed over the slowest rank's time."""
+    return world * bytes_per_rank / (ms * 1e-3) / 1e9
 
 
 def peaks():
@@ -200,12 +234,12 @@ def run_ours(args, rank, world, dist):
             step(False)
         t3.record(stream)
         torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
     ms = t2.elapsed_time(t3) / args.steps
     assert cache.status_flags() == 0, "device status flags set"
-    if dist:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(ms, dist, dev)
 
     # ---- algorithmic bytes
     nh = int(cache.n_high.sum().item())
@@ -229,7 +263,7 @@ def run_ours(args, rank, world, dist):
         hsh = hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read() for f in KERNEL_SOURCES)).hexdigest()
         if d.get("source_sha256") == hsh:
             traffic = d.get("dram_bytes_per_launch")
-    value = world * fp16_in / (ms * 1e-3) / 1e9
+    value = job_value(world, fp16_in, ms)
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
@@ -256,7 +290,7 @@ def run_ours(args, rank, world, dist):
     return res, (k, v, q_win, qdec, kn, vn, sn, seq_len, score, mask, out, cache, score_ws, fp16_in)
 
 
-def run_e2e(args, state):
+def run_e2e(args, state, dist=None):
     """Same step through the C ABI with pinned HOST inputs: H2D copies of K, V,
     the query window, the decode query and the new token inside the timed
     region, and a D2H read of the decode output."""
@@ -292,6 +326,9 @@ def run_e2e(args, state):
 
     for _ in range(2):
         step()
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
     torch.cuda.synchronize()
     n = max(2, min(args.steps, 5))
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -427,29 +464,18 @@ def main():
         return
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
-    dist = None
     if args.impl == "reference":
         res = run_reference(args, rank)
         if res is not None:
             print(json.dumps(res), flush=True)
         return
-    if world > 1:
-        import datetime
-
-        import torch
-        import torch.distributed as tdist
-        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", 0)))
-        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-        dist = tdist
+    rank, world, dist = init_ranks("nccl")
     res, state = run_ours(args, rank, world, dist)
     if not args.no_e2e:
-        e2e = run_e2e(args, state)
+        e2e = run_e2e(args, state, dist)
         if dist:
-            import torch
-            tt = torch.tensor([e2e["ms_per_step"]], device="cuda")
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e["ms_per_step"] = float(tt.item())
-            e2e["value"] = round(world * state[-1] / (e2e["ms_per_step"] * 1e-3) / 1e9, 2)
+            e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, "cuda")
+            e2e["value"] = round(job_value(world, state[-1], e2e["ms_per_step"]), 2)
         res["e2e"] = e2e
     if rank == 0 and world == 1 and not args.no_cpu:
         res["cpu_baseline"] = cpu_baseline_json()
