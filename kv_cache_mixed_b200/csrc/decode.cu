@@ -24,6 +24,13 @@
 // writes one partial (m, l, o[128]) per query head.  The FP16 block gets its
 // own small kernel and a last kernel merges all partials of a (sequence,
 // layer, KV head) into the output.
+//
+// MMA shapes per 16-token tile: the logits put the 16 tokens on the MMA rows
+// and the query heads on the 8 columns (one m16n8k16 per 16 head-dim slots);
+// the values put 16 head-dim slots on the rows and the query heads on the
+// columns, with P' moved into that operand layout by movmatrix.  With at most
+// 4 query heads per KV head, columns 4..7 of the value MMA carry the low f16
+// part of P', so one MMA takes both parts.
 #include "common.cuh"
 #include "internal.h"
 
@@ -211,7 +218,7 @@ constexpr int kWaitLimit = 1 << 20;         // mbarrier polls before a copy is d
 constexpr int kLutBytes = 64 * 4;           // pair table, L*L <= 36 entries
 
 template <int L>
-__global__ void __launch_bounds__(DEC_WARPS * 32)
+__global__ void __launch_bounds__(DEC_WARPS * 32, 4)
 decode_pool_kernel(const DecParams p) {
   using Gm = Geo<L>;
   constexpr int KB = Gm::KB, W = Gm::W;
@@ -265,6 +272,14 @@ decode_pool_kernel(const DecParams p) {
   qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
   const float qsc = qsum * p.c2;
   const float kscale = p.c2 * 16777216.0f;             // 2^24: codes are c * 2^-24
+  // This lane's two queries are the MMA columns 2c, 2c+1 of the logits.  With
+  // G <= 4 the value MMA's columns 4..7 carry the low f16 part of P' for
+  // queries 0..3, so lanes c >= 2 mirror the softmax of lane c-2 and one MMA
+  // per k-block takes both parts.
+  const bool pack_lo = G <= 4;
+  const int qc0 = pack_lo ? ((2 * c) & 3) : 2 * c;
+  const float qs0 = __shfl_sync(0xffffffffu, qsc, 4 * qc0);        // sum(q)*c2 lives in quad r
+  const float qs1 = __shfl_sync(0xffffffffu, qsc, 4 * (qc0 + 1));
 
   // ---- this CTA's tiles
   const int n = min(p.count[b], p.cap);
@@ -291,7 +306,7 @@ decode_pool_kernel(const DecParams p) {
     }
   };
 
-  float m_run = -INFINITY, l_run = 0.0f, mt_run = 0.0f;
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f}, mt_run[2] = {0.0f, 0.0f};
   float oacc[KB][4];
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) oacc[kb][0] = oacc[kb][1] = oacc[kb][2] = oacc[kb][3] = 0.0f;
@@ -322,34 +337,45 @@ decode_pool_kernel(const DecParams p) {
     const float2 *svm = reinterpret_cast<const float2 *>(tbuf + 128 * W + 128);
     const int t0 = tile * 16;
 
-    // ---- logits: S^T = Q C^T per 8-token group
-    float lg[2][2];
+    // ---- logits S = C Q^T: tokens r, r+8 on the MMA rows, queries on the
+    // columns; even and odd k-blocks accumulate apart (shorter MMA chain)
+    float lg[4];                          // (token r, q0), (r, q1), (r+8, q0), (r+8, q1)
+    {
+      uint32_t ka[KB][2], kb8[KB][2];
+      unpack_row<L>(sk + r * W, c, Lr, L2r, lut, ka);
+      unpack_row<L>(sk + (8 + r) * W, c, Lr, L2r, lut, kb8);
+      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int grp = 0; grp < 2; ++grp) {
-      uint32_t kr[KB][2];
-      unpack_row<L>(sk + (grp * 8 + r) * W, c, Lr, L2r, lut, kr);
-      float s[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int kb = 0; kb < KB; ++kb) {
+        if (kb & 1) mma_16816(sb, ka[kb][0], kb8[kb][0], ka[kb][1], kb8[kb][1], qa[kb][0], qa[kb][1]);
+        else mma_16816(sa, ka[kb][0], kb8[kb][0], ka[kb][1], kb8[kb][1], qa[kb][0], qa[kb][1]);
+      }
 #pragma unroll
-      for (int kb = 0; kb < KB; ++kb) mma_16816(s, qa[kb][0], 0u, qa[kb][1], 0u, kr[kb][0], kr[kb][1]);
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int tt = grp * 8 + 2 * c + e;
+      for (int i = 0; i < 4; ++i) {
+        float sv = sa[i] + sb[i];
+        const float mirror = __shfl_xor_sync(0xffffffffu, sv, 2);
+        if (pack_lo && c >= 2) sv = mirror;
+        const int tt = (i < 2) ? r : 8 + r;
         const float2 mm = skm[tt];
-        const float v = __fmaf_rn(s[e], mm.y * kscale, mm.x * qsc);
-        lg[grp][e] = (t0 + tt < n) ? v : -INFINITY;
+        const float v = __fmaf_rn(sv, mm.y * kscale, mm.x * ((i & 1) ? qs1 : qs0));
+        lg[i] = (t0 + tt < n) ? v : -INFINITY;
       }
     }
-    // ---- online softmax (log2 domain), query r per lane quad
-    float mx = fmaxf(fmaxf(lg[0][0], lg[0][1]), fmaxf(lg[1][0], lg[1][1]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m_run, mx);
-    if (__any_sync(0xffffffffu, m_new > m_run)) {
-      const float alpha = (m_new > m_run) ? ex2_approx(m_run - m_new) : 1.0f;   // m_run=-inf -> 0
-      l_run *= alpha;
-      mt_run *= alpha;
-      const float a0 = __shfl_sync(0xffffffffu, alpha, 8 * c);       // query 2c
-      const float a1 = __shfl_sync(0xffffffffu, alpha, 8 * c + 4);   // query 2c+1
+    // ---- online softmax (log2 domain): max over the 16 tokens = over r
+    float mx0 = fmaxf(lg[0], lg[2]), mx1 = fmaxf(lg[1], lg[3]);
+#pragma unroll
+    for (int o = 4; o <= 16; o <<= 1) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+    if (__any_sync(0xffffffffu, (mn0 > m_run[0]) | (mn1 > m_run[1]))) {
+      const float a0 = (mn0 > m_run[0]) ? ex2_approx(m_run[0] - mn0) : 1.0f;   // m_run=-inf -> 0
+      const float a1 = (mn1 > m_run[1]) ? ex2_approx(m_run[1] - mn1) : 1.0f;
+      l_run[0] *= a0;
+      mt_run[0] *= a0;
+      l_run[1] *= a1;
+      mt_run[1] *= a1;
 #pragma unroll
       for (int kb = 0; kb < KB; ++kb) {
         oacc[kb][0] *= a0;
@@ -357,45 +383,60 @@ decode_pool_kernel(const DecParams p) {
         oacc[kb][2] *= a0;
         oacc[kb][3] *= a1;
       }
-      m_run = m_new;
+      m_run[0] = mn0;
+      m_run[1] = mn1;
     }
     // P' = p * scale * kappa as an f16 pair hi + lo (hi = RN(P'), lo = RN(P' - hi)):
     // relative error 2^-22 instead of 2^-11 for a single f16
-    float pw[2][2];
+    uint32_t xh[2], xl[2];                // (token r | r+8): f16x2 of columns 2c, 2c+1
 #pragma unroll
-    for (int grp = 0; grp < 2; ++grp)
+    for (int g2 = 0; g2 < 2; ++g2) {
+      const int tt = g2 ? 8 + r : r;
+      const bool ok = t0 + tt < n;
+      const float2 vmm = svm[tt];
+      float pw[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int tt = grp * 8 + 2 * c + e;
-        const bool ok = t0 + tt < n;
-        const float pr = ok ? ex2_approx(lg[grp][e] - m_run) : 0.0f;
-        const float2 vmm = svm[tt];
-        l_run += pr;
-        mt_run += ok ? pr * vmm.x : 0.0f;
-        pw[grp][e] = ok ? pr * (vmm.y * kappa) : 0.0f;
+        const float pr = ok ? ex2_approx(lg[2 * g2 + e] - m_run[e]) : 0.0f;
+        l_run[e] += pr;
+        mt_run[e] += pr * vmm.x;
+        pw[e] = pr * (vmm.y * kappa);
       }
-    uint32_t bh[2], bl[2];
-#pragma unroll
-    for (int grp = 0; grp < 2; ++grp) {
-      const __half2 hi = __floats2half2_rn(pw[grp][0], pw[grp][1]);
+      const __half2 hi = __floats2half2_rn(pw[0], pw[1]);
       const float2 hf = __half22float2(hi);
-      const __half2 lo = __floats2half2_rn(pw[grp][0] - hf.x, pw[grp][1] - hf.y);
-      bh[grp] = *reinterpret_cast<const uint32_t *>(&hi);
-      bl[grp] = *reinterpret_cast<const uint32_t *>(&lo);
+      const __half2 lo = __floats2half2_rn(pw[0] - hf.x, pw[1] - hf.y);
+      xh[g2] = *reinterpret_cast<const uint32_t *>(&hi);
+      xl[g2] = *reinterpret_cast<const uint32_t *>(&lo);
     }
 
-    // ---- values: O^T += C^T P' (codes transposed in registers)
+    // ---- values: O^T += C^T P' (codes and P' transposed in registers)
     uint32_t vr0[KB][2], vr1[KB][2];
     unpack_row<L>(sv + r * W, c, Lr, L2r, lut, vr0);
     unpack_row<L>(sv + (8 + r) * W, c, Lr, L2r, lut, vr1);
+    if (pack_lo) {
+      // columns 0..3: hi parts (lanes c < 2), 4..7: lo parts (lanes c >= 2)
+      const uint32_t b0 = movmatrix_t(c < 2 ? xh[0] : xl[0]);
+      const uint32_t b1 = movmatrix_t(c < 2 ? xh[1] : xl[1]);
 #pragma unroll
-    for (int kb = 0; kb < KB; ++kb) {
-      const uint32_t a0 = movmatrix_t(vr0[kb][0]);
-      const uint32_t a1 = movmatrix_t(vr0[kb][1]);
-      const uint32_t a2 = movmatrix_t(vr1[kb][0]);
-      const uint32_t a3 = movmatrix_t(vr1[kb][1]);
-      mma_16816(oacc[kb], a0, a1, a2, a3, bh[0], bh[1]);
-      mma_16816(oacc[kb], a0, a1, a2, a3, bl[0], bl[1]);
+      for (int kb = 0; kb < KB; ++kb) {
+        const uint32_t a0 = movmatrix_t(vr0[kb][0]);
+        const uint32_t a1 = movmatrix_t(vr0[kb][1]);
+        const uint32_t a2 = movmatrix_t(vr1[kb][0]);
+        const uint32_t a3 = movmatrix_t(vr1[kb][1]);
+        mma_16816(oacc[kb], a0, a1, a2, a3, b0, b1);
+      }
+    } else {
+      const uint32_t bh0 = movmatrix_t(xh[0]), bh1 = movmatrix_t(xh[1]);
+      const uint32_t bl0 = movmatrix_t(xl[0]), bl1 = movmatrix_t(xl[1]);
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb) {
+        const uint32_t a0 = movmatrix_t(vr0[kb][0]);
+        const uint32_t a1 = movmatrix_t(vr0[kb][1]);
+        const uint32_t a2 = movmatrix_t(vr1[kb][0]);
+        const uint32_t a3 = movmatrix_t(vr1[kb][1]);
+        mma_16816(oacc[kb], a0, a1, a2, a3, bh0, bh1);
+        mma_16816(oacc[kb], a0, a1, a2, a3, bl0, bl1);
+      }
     }
     __syncwarp();
     slotix = (slotix + 1) % DEC_NST;
@@ -409,34 +450,48 @@ decode_pool_kernel(const DecParams p) {
       mbar_wait(&bars[s2], (parity >> s2) & 1u, kWaitLimit);
   }
 
-  // ---- quad totals of l and the min term (query r)
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
-  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
-  mt_run += __shfl_xor_sync(0xffffffffu, mt_run, 1);
-  mt_run += __shfl_xor_sync(0xffffffffu, mt_run, 2);
+  // ---- totals of l and of the min term over the token rows (lanes r); with
+  // packed low parts, lanes c >= 2 hold the low-part sums of queries 2c-4, 2c-3
+#pragma unroll
+  for (int o = 4; o <= 16; o <<= 1)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      l_run[e] += __shfl_xor_sync(0xffffffffu, l_run[e], o);
+      mt_run[e] += __shfl_xor_sync(0xffffffffu, mt_run[e], o);
+    }
+  if (pack_lo)
+#pragma unroll
+    for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) oacc[kb][i] += __shfl_xor_sync(0xffffffffu, oacc[kb][i], 2);
+  const bool owner = !pack_lo || c < 2;
 
   // ---- merge the 4 warps in shared memory (reuses the ring)
   __syncthreads();
   float *wo = reinterpret_cast<float *>(smem);                        // [warps][GMAX][128]
   float *wst = wo + DEC_WARPS * DEC_GMAX * kD;                        // [warps][GMAX][3]
-  if (c == 0 && r < G) {
-    wst[(warp * DEC_GMAX + r) * 3 + 0] = m_run;
-    wst[(warp * DEC_GMAX + r) * 3 + 1] = l_run;
-    wst[(warp * DEC_GMAX + r) * 3 + 2] = mt_run;
-  }
+  if (owner && r == 0)
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+      if (qc0 + e < G) {
+        wst[(warp * DEC_GMAX + qc0 + e) * 3 + 0] = m_run[e];
+        wst[(warp * DEC_GMAX + qc0 + e) * 3 + 1] = l_run[e];
+        wst[(warp * DEC_GMAX + qc0 + e) * 3 + 2] = mt_run[e];
+      }
   constexpr float unscale = 16777216.0f / kappa;
+  if (owner)
 #pragma unroll
-  for (int kb = 0; kb < KB; ++kb) {
+    for (int kb = 0; kb < KB; ++kb) {
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      // slot r (hh=0) or 8+r (hh=1) of block kb belongs to lane group r/2, position (r%2) + 2hh
-      const int d = slot_dim<L>(r >> 1, 4 * kb + 2 * hh + (r & 1));
-      if (d >= 0) {
-        if (2 * c < G) wo[(warp * DEC_GMAX + 2 * c) * kD + d] = oacc[kb][2 * hh] * unscale;
-        if (2 * c + 1 < G) wo[(warp * DEC_GMAX + 2 * c + 1) * kD + d] = oacc[kb][2 * hh + 1] * unscale;
+      for (int hh = 0; hh < 2; ++hh) {
+        // slot r (hh=0) or 8+r (hh=1) of block kb belongs to lane group r/2, position (r%2) + 2hh
+        const int d = slot_dim<L>(r >> 1, 4 * kb + 2 * hh + (r & 1));
+        if (d >= 0) {
+          if (qc0 < G) wo[(warp * DEC_GMAX + qc0) * kD + d] = oacc[kb][2 * hh] * unscale;
+          if (qc0 + 1 < G) wo[(warp * DEC_GMAX + qc0 + 1) * kD + d] = oacc[kb][2 * hh + 1] * unscale;
+        }
       }
     }
-  }
   __syncthreads();
   float *dst = p.part + ((int64_t)slab * p.NU + p.unit0 + split) * G * PART_STRIDE;
   for (int i = threadIdx.x; i < G * kD; i += DEC_WARPS * 32) {

@@ -115,6 +115,26 @@ def test_levels_quantize_and_decode(L_high, L_low):
     check_attention(to_np(out), ref)
 
 
+# query heads per KV head: 1..3 leave MMA columns unused, 4 packs the low f16
+# part of P' into the free columns, 6 and 8 use every column
+@pytest.mark.parametrize("H,H_q", [(2, 2), (2, 4), (1, 3), (2, 8), (2, 12), (1, 8)])
+def test_decode_gqa_group_sizes(H, H_q):
+    kv = kv_mod()
+    wl = synth.scaled(synth.TINY, B=2, Lyr=2, H=H, H_q=H_q, T=333)
+    k, v = synth.kv(wl, 40 + H_q, DEV)
+    score = synth.uniform_score(wl, H_q, DEV)
+    seq_len = torch.tensor([333, 201], dtype=torch.int32, device=DEV)
+    cache, mask = _prefill(k, v, score, seq_len, 6, 5, 500_000, wl.H_q)
+    masks = _oracle_masks(score, [333, 201], 500_000)
+    assert _status(cache) == 0
+    kn, vn = to_np(k), to_np(v)
+    q = synth.decode_query(wl, 5, DEV)
+    out = torch.empty_like(q)
+    kv.semkv_decode_attn(cache, 0, 2, q, out)
+    ref = _oracle_decode_slabs(kn, vn, masks, [333, 201], to_np(q), 6, 5)
+    check_attention(to_np(out), ref)
+
+
 # ----------------------------------------------------------------- adversarial rows
 def _adversarial_rows(rng, n):
     rows = []
