@@ -581,28 +581,29 @@ __global__ void __launch_bounds__(128) decode_buffer_kernel(const BufParams p) {
   }
 }
 
-// ---- merge all partials of a (sequence, layer, KV head): thread = head dim
+// ---- merge all partials of a (sequence, layer, KV head) for one query head:
+// CTA = (slab, query head of the group), thread = head dim
 __global__ void __launch_bounds__(128) decode_merge_kernel(const float *__restrict__ part, int NU,
                                                            int G, int H, int nL, int H_q,
                                                            uint16_t *__restrict__ out) {
-  const int slab = blockIdx.x, d = threadIdx.x;
+  const int slab = blockIdx.x / G, qh = blockIdx.x % G, d = threadIdx.x;
   const int h = slab % H, li = (slab / H) % nL, b = slab / (H * nL);
-  for (int qh = 0; qh < G; ++qh) {
-    float M = -INFINITY;
-    for (int u = 0; u < NU; ++u) M = fmaxf(M, part[((int64_t)slab * NU + u) * G * PART_STRIDE + qh * PART_STRIDE]);
-    float o = 0.0f, l = 0.0f;
-    if (M != -INFINITY) {
-      for (int u = 0; u < NU; ++u) {
-        const float *pp = part + ((int64_t)slab * NU + u) * G * PART_STRIDE + qh * PART_STRIDE;
-        if (pp[0] == -INFINITY) continue;
-        const float a = ex2_approx(pp[0] - M);
-        o += a * pp[4 + d];
-        l += a * pp[1];
-      }
+  const float *pq = part + (int64_t)slab * NU * G * PART_STRIDE + qh * PART_STRIDE;
+  float M = -INFINITY;
+  for (int u = 0; u < NU; ++u) M = fmaxf(M, pq[(int64_t)u * G * PART_STRIDE]);
+  float o = 0.0f, l = 0.0f;
+  if (M != -INFINITY) {
+    for (int u = 0; u < NU; ++u) {
+      const float *pp = pq + (int64_t)u * G * PART_STRIDE;
+      const float mu = pp[0];
+      if (mu == -INFINITY) continue;
+      const float a = ex2_approx(mu - M);
+      o += a * pp[4 + d];
+      l += a * pp[1];
     }
-    const float res = l > 0.0f ? o / l : 0.0f;
-    out[(((int64_t)b * nL + li) * H_q + h * G + qh) * kD + d] = __half_as_ushort(__float2half_rn(res));
   }
+  const float res = l > 0.0f ? o / l : 0.0f;
+  out[(((int64_t)b * nL + li) * H_q + h * G + qh) * kD + d] = __half_as_ushort(__float2half_rn(res));
 }
 
 // ---------------------------------------------------------------- host side
@@ -714,7 +715,7 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, const 
   decode_buffer_kernel<<<slabs, 128, 0, st>>>(bp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_merge_kernel<<<slabs, 128, 0, st>>>(p.part, NU, G, c.H, n_layers, c.H_q, out);
+  decode_merge_kernel<<<slabs * G, 128, 0, st>>>(p.part, NU, G, c.H, n_layers, c.H_q, out);
   return cudaGetLastError();
 }
 

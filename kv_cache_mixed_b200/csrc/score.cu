@@ -265,19 +265,27 @@ __global__ void __launch_bounds__(AM_WARPS * 32, 1) attn_rowstats_kernel(const A
     }
 }
 
-// merge pass-1 partials: one thread per window row
-__global__ void attn_merge_kernel(const AttnParams p) {
-  const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+// merge pass-1 partials: one warp per window row, lanes over the T chunks
+// (nchunk <= 64), reduced by a fixed shuffle tree
+__global__ void __launch_bounds__(256) attn_merge_kernel(const AttnParams p) {
+  const int64_t row = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   const int64_t nrows = (int64_t)p.B * p.H_q * p.w;
-  if (idx >= nrows) return;
-  const float2 *pp = p.part + idx * p.nchunk;
-  float M = -INFINITY;
-  for (int c = 0; c < p.nchunk; ++c) M = fmaxf(M, pp[c].x);
+  if (row >= nrows) return;
+  const float2 *pp = p.part + row * p.nchunk;
+  const float2 a = lane < p.nchunk ? pp[lane] : make_float2(-INFINITY, 0.0f);
+  const float2 c = lane + 32 < p.nchunk ? pp[lane + 32] : make_float2(-INFINITY, 0.0f);
+  float M = fmaxf(a.x, c.x);
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float Z = 0.0f;
-  if (M != -INFINITY)
-    for (int c = 0; c < p.nchunk; ++c)
-      if (pp[c].x != -INFINITY) Z += pp[c].y * ex2_approx(pp[c].x - M);
-  p.stats[idx] = make_float2(M, Z > 0.0f ? 1.0f / Z : 0.0f);
+  if (M != -INFINITY) {
+    if (a.x != -INFINITY) Z += a.y * ex2_approx(a.x - M);
+    if (c.x != -INFINITY) Z += c.y * ex2_approx(c.x - M);
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
+  if (lane == 0) p.stats[row] = make_float2(M, Z > 0.0f ? 1.0f / Z : 0.0f);
 }
 
 // pass 2: grid (ceil(T_max/64), B); each CTA sums 64 key columns over every
@@ -683,7 +691,7 @@ cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const u
     attn_umma_kernel<1><<<dim3(nch, H, B), UA_THREADS, UA_SMEM, st>>>(p, Np, nch, head_part);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_merge_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
+    attn_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_umma_kernel<2><<<dim3(nch, H, B), UA_THREADS, UA_SMEM, st>>>(p, Np, nch, head_part);
@@ -698,7 +706,7 @@ cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const u
   attn_rowstats_kernel<<<dim3(p.nchunk, H * p.nrb, B), AM_WARPS * 32, 0, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  attn_merge_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, st>>>(p);
+  attn_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   attn_colsum_kernel<<<dim3(ntile, B), AM_WARPS * 32, 0, st>>>(p);
