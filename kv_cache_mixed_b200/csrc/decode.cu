@@ -216,6 +216,8 @@ static_assert(Geo<6>::TILE_BYTES % 16 == 0 && Geo<5>::TILE_BYTES % 16 == 0 && kM
               "tile buffers must keep 16-byte alignment for bulk copies");
 constexpr int kWaitLimit = 1 << 20;         // mbarrier polls before a copy is declared lost
 constexpr int kLutBytes = 64 * 4;           // pair table, L*L <= 36 entries
+template <int L>
+constexpr int kQfragBytes = Geo<L>::KB * 32 * 8;   // q operand fragments, [kb][lane] x 2 words
 
 template <int L>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 4)
@@ -236,7 +238,8 @@ decode_pool_kernel(const DecParams p) {
   uint8_t *ring = smem + warp * DEC_NST * Gm::TILE_BYTES;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff<L>) + warp * DEC_NST;
   uint32_t *lut = reinterpret_cast<uint32_t *>(smem + kQOff<L>);      // [L*L] digit pairs (pair path)
-  float *qs = reinterpret_cast<float *>(smem + kQOff<L> + kLutBytes);  // [G][128]
+  uint2 *qfrag = reinterpret_cast<uint2 *>(smem + kQOff<L> + kLutBytes);            // [KB][32]
+  float *qs = reinterpret_cast<float *>(smem + kQOff<L> + kLutBytes + kQfragBytes<L>);  // [G][128]
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < DEC_NST; ++s) mbar_init(&bars[s], 1);
@@ -251,11 +254,12 @@ decode_pool_kernel(const DecParams p) {
   }
   __syncthreads();
 
-  // ---- q fragments in slot order, and sum(q) * c2 for this lane's query r
-  uint32_t qa[KB][2];
+  // ---- q fragments in slot order (kept in shared memory, one copy per CTA:
+  // every warp uses the same fragments), and sum(q) * c2 for this lane's query r
   float qsum = 0.0f;
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) {
+    uint32_t qv[2];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float v[2];
@@ -265,9 +269,11 @@ decode_pool_kernel(const DecParams p) {
         v[e] = (r < G && d >= 0) ? qs[r * kD + d] : 0.0f;
         qsum += v[e];
       }
-      qa[kb][hh] = pack_half2(v[0], v[1]);
+      qv[hh] = pack_half2(v[0], v[1]);
     }
+    if (warp == 0) qfrag[kb * 32 + lane] = make_uint2(qv[0], qv[1]);
   }
+  __syncthreads();
   qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
   qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
   const float qsc = qsum * p.c2;
@@ -347,8 +353,9 @@ decode_pool_kernel(const DecParams p) {
       float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int kb = 0; kb < KB; ++kb) {
-        if (kb & 1) mma_16816(sb, ka[kb][0], kb8[kb][0], ka[kb][1], kb8[kb][1], qa[kb][0], qa[kb][1]);
-        else mma_16816(sa, ka[kb][0], kb8[kb][0], ka[kb][1], kb8[kb][1], qa[kb][0], qa[kb][1]);
+        const uint2 qb = qfrag[kb * 32 + lane];
+        if (kb & 1) mma_16816(sb, ka[kb][0], kb8[kb][0], ka[kb][1], kb8[kb][1], qb.x, qb.y);
+        else mma_16816(sa, ka[kb][0], kb8[kb][0], ka[kb][1], kb8[kb][1], qb.x, qb.y);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -609,7 +616,7 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float *__restri
 // ---------------------------------------------------------------- host side
 template <int L>
 static int pool_smem_bytes(int G) {
-  return kQOff<L> + kLutBytes + G * kD * 4;
+  return kQOff<L> + kLutBytes + kQfragBytes<L> + G * kD * 4;
 }
 
 template <int L>
