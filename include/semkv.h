@@ -238,6 +238,23 @@ semkv_status semkv_decode_attn(const semkv_cache *c, int32_t layer0, int32_t n_l
                                const uint16_t *q, uint16_t *out, float sm_scale, void *ws,
                                size_t ws_bytes, uint32_t *status, void *stream);
 
+/*
+ * semkv_decode_attn plus the attention-mass indicator for generated tokens
+ * (SemKV, Fig. 6: the scores of generated tokens are accumulated until their
+ * block is ranked; Fig. 12: attention-based indicators).  At the scoring layer
+ * score_layer (layer0 <= score_layer < layer0 + n_layers), every FP16-block
+ * token t < buf_len receives, in buf_score[b][t], the sum over the H_q query
+ * heads of its softmax probability in this step, normalised over every cached
+ * token exactly as the output is.  Heads are added in index order, so the
+ * result is deterministic.  The block's ranking in semkv_append_block then
+ * uses these accumulated scores (plus whatever score_new the caller gave).
+ * Same workspace as semkv_decode_attn.  Errors: as semkv_decode_attn, plus
+ * INVALID_ARG for score_layer outside the decoded layers or a null buf_score.
+ */
+semkv_status semkv_decode_attn_acc(const semkv_cache *c, int32_t layer0, int32_t n_layers,
+                                   int32_t score_layer, const uint16_t *q, uint16_t *out, float sm_scale,
+                                   void *ws, size_t ws_bytes, uint32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

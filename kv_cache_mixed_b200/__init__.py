@@ -6,6 +6,6 @@ has not been built (`python kv_cache_mixed_b200/build.py`).
 """
 from .binding import (FLAG_CAPACITY, FLAG_NONFINITE, FLAG_SEQLEN, FLUSH, SCORE_ATTN_MASS,  # noqa: F401
                       SCORE_KEY_L2, EXPORTED, LIB_PATH, MixedCache, SemkvError, semkv_append_block,
-                      semkv_decode_attn, semkv_digits_per_word, semkv_num_high, semkv_quantize,
+                      semkv_decode_attn, semkv_decode_attn_acc, semkv_digits_per_word, semkv_num_high, semkv_quantize,
                       semkv_quantize_noalloc, semkv_score, semkv_select, semkv_version,
                       semkv_words_per_row)

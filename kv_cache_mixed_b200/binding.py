@@ -65,12 +65,14 @@ _lib_append = _sig("semkv_append_block", _i32, [ctypes.POINTER(SemkvCache), _p, 
 _lib_decode_ws = _sig("semkv_decode_workspace_size", _sz, [ctypes.POINTER(SemkvCache), _i32])
 _lib_decode = _sig("semkv_decode_attn", _i32, [ctypes.POINTER(SemkvCache), _i32, _i32, _p, _p, _f32, _p, _sz, _p,
                                                 _p])
+_lib_decode_acc = _sig("semkv_decode_attn_acc", _i32, [ctypes.POINTER(SemkvCache), _i32, _i32, _i32, _p, _p, _f32,
+                                                      _p, _sz, _p, _p])
 
 EXPORTED = ["semkv_num_high", "semkv_digits_per_word", "semkv_words_per_row", "semkv_version",
             "semkv_score_workspace_size", "semkv_score", "semkv_select_workspace_size", "semkv_select",
             "semkv_quantize_workspace_size", "semkv_quantize", "semkv_quantize_noalloc",
             "semkv_append_workspace_size",
-            "semkv_append_block", "semkv_decode_workspace_size", "semkv_decode_attn"]
+            "semkv_append_block", "semkv_decode_workspace_size", "semkv_decode_attn", "semkv_decode_attn_acc"]
 
 
 class SemkvError(RuntimeError):
@@ -225,4 +227,13 @@ def semkv_decode_attn(cache: MixedCache, layer0: int, n_layers: int, q: torch.Te
     ws = cache.workspace(("decode", n_layers), int(_lib_decode_ws(ctypes.byref(cache.c), n_layers)))
     _check(_lib_decode(ctypes.byref(cache.c), layer0, n_layers, _ptr(q), _ptr(out), sm_scale, _ptr(ws),
                        ws.numel(), _ptr(cache.status), _stream(stream)), "semkv_decode_attn")
+    return out
+
+
+def semkv_decode_attn_acc(cache: MixedCache, layer0: int, n_layers: int, score_layer: int, q: torch.Tensor,
+                          out: torch.Tensor, sm_scale: float = 128 ** -0.5, stream=None):
+    """semkv_decode_attn, and the FP16 block's attention mass at score_layer added into cache.buf_score."""
+    ws = cache.workspace(("decode", n_layers), int(_lib_decode_ws(ctypes.byref(cache.c), n_layers)))
+    _check(_lib_decode_acc(ctypes.byref(cache.c), layer0, n_layers, score_layer, _ptr(q), _ptr(out), sm_scale,
+                           _ptr(ws), ws.numel(), _ptr(cache.status), _stream(stream)), "semkv_decode_attn_acc")
     return out

@@ -222,16 +222,30 @@ size_t semkv_decode_workspace_size(const semkv_cache *c, int32_t n_layers) {
   return decode_ws_bytes(*c, n_layers);
 }
 
-semkv_status semkv_decode_attn(const semkv_cache *c, int32_t layer0, int32_t n_layers,
-                               const uint16_t *q, uint16_t *out, float sm_scale, void *ws,
-                               size_t ws_bytes, uint32_t *status, void *stream) {
+static semkv_status decode_checked(const semkv_cache *c, int32_t layer0, int32_t n_layers, int32_t score_layer,
+                                   const uint16_t *q, uint16_t *out, float sm_scale, void *ws,
+                                   size_t ws_bytes, uint32_t *status, void *stream) {
   semkv_status s = check_cache(c);
   if (s != SEMKV_OK) return s;
   if (layer0 < 0 || n_layers <= 0 || layer0 + n_layers > c->n_layers) return SEMKV_ERR_INVALID_ARG;
   if (!al16(q) || !al16(out)) return SEMKV_ERR_INVALID_ARG;
   if (!(sm_scale > 0.0f) || sm_scale != sm_scale) return SEMKV_ERR_INVALID_ARG;
   if (!al16(ws) || ws_bytes < decode_ws_bytes(*c, n_layers)) return SEMKV_ERR_WORKSPACE;
-  return cuda_status(launch_decode(*c, layer0, n_layers, q, out, sm_scale, ws, status, S(stream)));
+  return cuda_status(launch_decode(*c, layer0, n_layers, score_layer, q, out, sm_scale, ws, status, S(stream)));
+}
+
+semkv_status semkv_decode_attn(const semkv_cache *c, int32_t layer0, int32_t n_layers,
+                               const uint16_t *q, uint16_t *out, float sm_scale, void *ws,
+                               size_t ws_bytes, uint32_t *status, void *stream) {
+  return decode_checked(c, layer0, n_layers, -1, q, out, sm_scale, ws, ws_bytes, status, stream);
+}
+
+semkv_status semkv_decode_attn_acc(const semkv_cache *c, int32_t layer0, int32_t n_layers,
+                                   int32_t score_layer, const uint16_t *q, uint16_t *out, float sm_scale,
+                                   void *ws, size_t ws_bytes, uint32_t *status, void *stream) {
+  if (c && (score_layer < layer0 || score_layer >= layer0 + n_layers)) return SEMKV_ERR_INVALID_ARG;
+  if (c && c->buf_score == nullptr) return SEMKV_ERR_INVALID_ARG;
+  return decode_checked(c, layer0, n_layers, score_layer, q, out, sm_scale, ws, ws_bytes, status, stream);
 }
 
 }  // extern "C"

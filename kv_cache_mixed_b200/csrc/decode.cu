@@ -534,6 +534,8 @@ struct BufParams {
   float c2;
   float *part;
   int NU, unit;
+  int score_li;                // layer (relative to layer0) whose buffer logits are kept, or -1
+  float *logit;                // [B][H_q][block] log2-domain logits of the FP16 tokens
 };
 
 __global__ void __launch_bounds__(128) decode_buffer_kernel(const BufParams p) {
@@ -555,6 +557,7 @@ __global__ void __launch_bounds__(128) decode_buffer_kernel(const BufParams p) {
       float acc = 0.0f;
       for (int d = 0; d < kD; ++d) acc = fmaf(qs[qh][d], __half2float(__ushort_as_half(kb[(int64_t)tid * kD + d])), acc);
       sc[qh][tid] = acc * p.c2;
+      if (li == p.score_li) p.logit[((int64_t)b * p.H_q + h * G + qh) * p.block + tid] = acc * p.c2;
     }
   }
   __syncthreads();
@@ -589,10 +592,18 @@ __global__ void __launch_bounds__(128) decode_buffer_kernel(const BufParams p) {
 }
 
 // ---- merge all partials of a (sequence, layer, KV head) for one query head:
-// CTA = (slab, query head of the group), thread = head dim
+// CTA = (slab, query head of the group), thread = head dim.  At the scoring
+// layer, thread t < buf_len also writes the final softmax probability of
+// FP16 token t (same normalisation as the output) for the score accumulation.
+struct MergeAcc {
+  int score_li, block, buf_len;
+  const float *logit;          // [B][H_q][block]
+  float *prob;                 // [B][H_q][block]
+};
+
 __global__ void __launch_bounds__(128) decode_merge_kernel(const float *__restrict__ part, int NU,
                                                            int G, int H, int nL, int H_q,
-                                                           uint16_t *__restrict__ out) {
+                                                           uint16_t *__restrict__ out, const MergeAcc acc) {
   const int slab = blockIdx.x / G, qh = blockIdx.x % G, d = threadIdx.x;
   const int h = slab % H, li = (slab / H) % nL, b = slab / (H * nL);
   const float *pq = part + (int64_t)slab * NU * G * PART_STRIDE + qh * PART_STRIDE;
@@ -611,6 +622,21 @@ __global__ void __launch_bounds__(128) decode_merge_kernel(const float *__restri
   }
   const float res = l > 0.0f ? o / l : 0.0f;
   out[(((int64_t)b * nL + li) * H_q + h * G + qh) * kD + d] = __half_as_ushort(__float2half_rn(res));
+  if (li == acc.score_li && d < acc.buf_len) {
+    const int64_t ix = ((int64_t)b * H_q + h * G + qh) * acc.block + d;
+    acc.prob[ix] = (l > 0.0f) ? ex2_approx(acc.logit[ix] - M) / l : 0.0f;
+  }
+}
+
+// buf_score[b][t] += sum over the query heads, in order, of the probabilities
+// of FP16 token t at the scoring layer
+__global__ void decode_score_acc_kernel(const float *__restrict__ prob, int H_q, int block, int buf_len,
+                                        float *__restrict__ buf_score) {
+  const int b = blockIdx.x, t = threadIdx.x;
+  if (t >= buf_len) return;
+  float s = 0.0f;
+  for (int j = 0; j < H_q; ++j) s += prob[((int64_t)b * H_q + j) * block + t];
+  buf_score[(int64_t)b * block + t] += s;
 }
 
 // ---------------------------------------------------------------- host side
@@ -676,10 +702,11 @@ size_t decode_ws_bytes(const semkv_cache &c, int n_layers) {
   const int Sh = pool_splits(c, n_layers, c.cap_high), Sl = pool_splits(c, n_layers, c.cap_low);
   const int64_t slabs = (int64_t)c.B * n_layers * c.H;
   const int G = c.H_q / c.H;
-  return (size_t)(slabs * (Sh + Sl + 1) * G * PART_STRIDE * sizeof(float));
+  const size_t parts = (size_t)(slabs * (Sh + Sl + 1) * G * PART_STRIDE * sizeof(float));
+  return parts + 2 * (size_t)c.B * c.H_q * c.block * sizeof(float);
 }
 
-cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, const uint16_t *q,
+cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int score_layer, const uint16_t *q,
                           uint16_t *out, float sm_scale, void *ws, uint32_t *status, cudaStream_t st) {
   const int Sh = pool_splits(c, n_layers, c.cap_high), Sl = pool_splits(c, n_layers, c.cap_low);
   const int NU = Sh + Sl + 1;
@@ -719,10 +746,27 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, const 
   bp.B = c.B; bp.Lyr = c.n_layers; bp.H = c.H; bp.H_q = c.H_q; bp.G = G;
   bp.layer0 = layer0; bp.nL = n_layers; bp.q = q; bp.c2 = p.c2;
   bp.part = p.part; bp.NU = NU; bp.unit = Sh + Sl;
+  // score accumulation at the scoring layer (relative index, -1 = none)
+  const int score_li = (score_layer >= layer0 && score_layer < layer0 + n_layers && c.buf_len > 0)
+                           ? score_layer - layer0 : -1;
+  float *logit = reinterpret_cast<float *>(reinterpret_cast<char *>(ws) +
+                                           (size_t)slabs * NU * G * PART_STRIDE * sizeof(float));
+  float *prob = logit + (size_t)c.B * c.H_q * c.block;
+  bp.score_li = score_li;
+  bp.logit = logit;
   decode_buffer_kernel<<<slabs, 128, 0, st>>>(bp);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_merge_kernel<<<slabs * G, 128, 0, st>>>(p.part, NU, G, c.H, n_layers, c.H_q, out);
+  MergeAcc ma;
+  ma.score_li = score_li;
+  ma.block = c.block;
+  ma.buf_len = c.buf_len;
+  ma.logit = logit;
+  ma.prob = prob;
+  decode_merge_kernel<<<slabs * G, 128, 0, st>>>(p.part, NU, G, c.H, n_layers, c.H_q, out, ma);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || score_li < 0) return e;
+  decode_score_acc_kernel<<<c.B, c.block, 0, st>>>(prob, c.H_q, c.block, c.buf_len, c.buf_score);
   return cudaGetLastError();
 }
 

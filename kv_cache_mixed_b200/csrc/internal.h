@@ -50,7 +50,7 @@ cudaError_t launch_buffer_append(const semkv_cache &c, const uint16_t *k_new,
                                  int i0, int take, cudaStream_t st);
 
 size_t decode_ws_bytes(const semkv_cache &c, int n_layers);
-cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, const uint16_t *q,
+cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int score_layer, const uint16_t *q,
                           uint16_t *out, float sm_scale, void *ws, uint32_t *status, cudaStream_t st);
 
 }  // namespace semkv

@@ -361,8 +361,11 @@ class MixedCache:
                     np.concatenate([p.mn for p in parts]),
                     np.concatenate([p.scale for p in parts]))
 
-    def decode(self, q, sm_scale=None, layer0=0):
-        """GQA decode attention over the mixed cache, float64 (see decode_attn)."""
+    def decode(self, q, sm_scale=None, layer0=0, score_layer=None):
+        """GQA decode attention over the mixed cache, float64 (see decode_attn).
+
+        With score_layer set, the FP16 block's tokens also accumulate the
+        attention they receive at that layer (see buffer_attention_mass)."""
         B, nL, H_q, D = q.shape
         out = np.zeros((B, nL, H_q, D), dtype=np.float64)
         for b in range(B):
@@ -384,6 +387,10 @@ class MixedCache:
                     keys.append(np.concatenate(kk))
                     vals.append(np.concatenate(vv))
                 out[b, li] = decode_attn(q[b, li], keys, vals, sm_scale)
+                nb = self.buf_k.shape[3]
+                if score_layer is not None and l == score_layer and nb > 0:
+                    mass = buffer_attention_mass(q[b, li], keys, nb, sm_scale)
+                    self.buf_score[b] = (self.buf_score[b].astype(np.float64) + mass).astype(np.float32)
         return out
 
 
@@ -412,6 +419,30 @@ def decode_attn(q: np.ndarray, keys: list, vals: list, sm_scale=None) -> np.ndar
         p = e / e.sum()
         out[h] = p @ vals[g]
     return out
+
+
+def buffer_attention_mass(q: np.ndarray, keys: list, n_buf: int, sm_scale=None) -> np.ndarray:
+    """Attention mass of the FP16-block tokens in one decode step, float64.
+
+    SemKV, Fig. 6: generated tokens wait in the FP16 block and their scores
+    are accumulated until the block is ranked; Fig. 12: attention-based
+    indicators.  Reading: at the scoring layer, token t of the block receives
+    sum over the H_q query heads of its softmax probability, normalised over
+    every cached token of the head's KV head (pools and block), i.e. the same
+    probabilities decode_attn uses.  keys[g] ends with the n_buf block tokens.
+    """
+    H_q, D = q.shape
+    H = len(keys)
+    G = H_q // H
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(D)
+    mass = np.zeros(n_buf, dtype=np.float64)
+    for h in range(H_q):
+        k = keys[h // G]
+        logits = (k @ q[h].astype(np.float64)) * sm_scale
+        e = np.exp(logits - logits.max())
+        mass += (e / e.sum())[k.shape[0] - n_buf:]
+    return mass
 
 
 # ---------------------------------------------------------------------------

@@ -387,6 +387,84 @@ def test_generation_block_exact(block, chunk):
     check_attention(to_np(out), ref.decode(q))
 
 
+@pytest.mark.parametrize("block", [16, 128])
+def test_generation_attention_mass_accumulation(block):
+    """Scores of generated tokens from the attention they receive at the scoring
+    layer: buf_score matches the oracle within the score tolerance after every
+    step, and each block is ranked on the GPU's accumulated scores (the oracle
+    takes the GPU score vector at the ranking, as for prefill), so every pool
+    row stays bit-exact."""
+    kv = kv_mod()
+    rng = np.random.default_rng(90 + block)
+    B, Lyr, H, H_q = 2, 2, 2, 8
+    lens = [70, 45]
+    T = max(lens)
+    L_high, L_low, r_ppm = 6, 5, 500_000
+    k = rng.standard_normal((B, Lyr, H, T, 128)).astype(np.float16)
+    v = rng.standard_normal((B, Lyr, H, T, 128)).astype(np.float16)
+    sc = rng.random((B, T)).astype(np.float32)
+    steps = block + 9
+    score_layer = Lyr - 1
+    cache, _ = _prefill(torch.from_numpy(k).to(DEV), torch.from_numpy(v).to(DEV), torch.from_numpy(sc).to(DEV),
+                        torch.tensor(lens, dtype=torch.int32, device=DEV), L_high, L_low, r_ppm, H_q,
+                        block=block, gen=steps)
+    ref = O.MixedCache(B, Lyr, H, L_high, L_low, r_ppm, block=block)
+    ref.prefill(k, v, lens, _oracle_masks(torch.from_numpy(sc), lens, r_ppm))
+    zeros = np.zeros((B, 1), np.float32)
+    for step in range(steps):
+        kn = rng.standard_normal((B, Lyr, H, 1, 128)).astype(np.float16)
+        vn = rng.standard_normal((B, Lyr, H, 1, 128)).astype(np.float16)
+        if ref.buf_k.shape[3] == block - 1:
+            # this append completes the block: rank it on the GPU's scores
+            ref.buf_score = to_np(cache.buf_score)[:, :block - 1].copy()
+        kv.semkv_append_block(cache, torch.from_numpy(kn).to(DEV), torch.from_numpy(vn).to(DEV),
+                              torch.from_numpy(zeros).to(DEV), 1)
+        ref.append(kn, vn, zeros)
+        q = rng.standard_normal((B, Lyr, H_q, 128)).astype(np.float16)
+        out = torch.empty((B, Lyr, H_q, 128), dtype=torch.float16, device=DEV)
+        kv.semkv_decode_attn_acc(cache, 0, Lyr, score_layer, torch.from_numpy(q).to(DEV), out)
+        check_attention(to_np(out), ref.decode(q, score_layer=score_layer))
+        nb = cache.buf_len
+        assert nb == ref.buf_k.shape[3]
+        gs = to_np(cache.buf_score)[:, :nb].astype(np.float64)
+        rs = ref.buf_score.astype(np.float64)
+        assert np.all(np.abs(gs - rs) <= SCORE_RTOL * np.abs(rs) + SCORE_ATOL), step
+    assert _status(cache) == 0
+    assert to_np(cache.n_high).tolist() == ref.n_high.tolist()
+    for b in range(B):
+        for l in range(Lyr):
+            for h in range(H):
+                for which, words in (("kh", cache.k_high), ("kl", cache.k_low), ("vh", cache.v_high),
+                                     ("vl", cache.v_low)):
+                    p = ref.pools(b, l, h, which)
+                    n = p.words.shape[0]
+                    assert np.array_equal(to_np(words[b, l, h, :n]).view(np.uint32), p.words)
+
+
+def test_decode_attn_acc_is_deterministic_and_matches_plain_decode():
+    kv = kv_mod()
+    rng = np.random.default_rng(77)
+    B, Lyr, H, H_q, T = 1, 2, 2, 8, 200
+    k = torch.from_numpy(rng.standard_normal((B, Lyr, H, T, 128)).astype(np.float16)).to(DEV)
+    sc = torch.from_numpy(rng.random((B, T)).astype(np.float32)).to(DEV)
+    cache, _ = _prefill(k, k, sc, torch.tensor([T], dtype=torch.int32, device=DEV), 6, 5, 500_000, H_q, gen=64)
+    kn = torch.from_numpy(rng.standard_normal((B, Lyr, H, 50, 128)).astype(np.float16)).to(DEV)
+    kv.semkv_append_block(cache, kn, kn, torch.zeros((B, 50), device=DEV), 50)
+    q = torch.from_numpy(rng.standard_normal((B, Lyr, H_q, 128)).astype(np.float16)).to(DEV)
+    o1, o2 = torch.empty_like(q), torch.empty_like(q)
+    kv.semkv_decode_attn(cache, 0, Lyr, q, o1)
+    s0 = cache.buf_score.clone()
+    kv.semkv_decode_attn_acc(cache, 0, Lyr, 0, q, o2)
+    assert torch.equal(o1, o2)                                        # same outputs
+    d1 = cache.buf_score - s0
+    cache.buf_score.copy_(s0)
+    kv.semkv_decode_attn_acc(cache, 0, Lyr, 0, q, o2)
+    assert torch.equal(cache.buf_score - s0, d1)                      # bitwise deterministic
+    assert float(d1[0, 50:].abs().max()) == 0.0                       # only the 50 block tokens
+    with pytest.raises(kv.SemkvError):
+        kv.semkv_decode_attn_acc(cache, 0, 1, 1, q[:, :1].contiguous(), o2[:, :1].contiguous())
+
+
 def test_decode_layer_subset_and_empty_sequence():
     kv = kv_mod()
     rng = np.random.default_rng(21)

@@ -359,6 +359,46 @@ def test_decode_all_fp16_buffer_is_textbook_attention():
     assert np.allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
 
 
+def test_buffer_mass_all_fp16_cache_sums_to_query_heads_and_matches_scipy():
+    # every key in the FP16 block: each head's probabilities sum to 1, and the
+    # mass equals scipy's softmax summed over the heads of each KV head
+    rng = np.random.default_rng(21)
+    B, Lyr, H, H_q, n = 2, 2, 2, 8, 37
+    cache = O.MixedCache(B, Lyr, H, 6, 5, 500_000)
+    kn = rng.standard_normal((B, Lyr, H, n, 128)).astype(np.float16)
+    cache.append(kn, kn, np.zeros((B, n), np.float32))
+    q = rng.standard_normal((B, Lyr, H_q, 128)).astype(np.float16)
+    cache.decode(q, score_layer=1)
+    for b in range(B):
+        assert abs(float(cache.buf_score[b].astype(np.float64).sum()) - H_q) < 1e-4
+        ref = np.zeros(n)
+        for h in range(H_q):
+            lg = kn[b, 1, h // (H_q // H)].astype(np.float64) @ q[b, 1, h].astype(np.float64) / math.sqrt(128)
+            ref += scipy.special.softmax(lg)
+        assert np.allclose(cache.buf_score[b], ref, rtol=1e-6, atol=1e-7)
+    # a second step accumulates; a step at another layer adds nothing
+    before = cache.buf_score.copy()
+    cache.decode(q, score_layer=1)
+    assert np.allclose(cache.buf_score, 2 * before.astype(np.float64), rtol=1e-6)
+    cache.decode(q, score_layer=None)
+    cache.decode(q[:, :1], layer0=0, score_layer=1)            # layer 1 not decoded: no change
+    assert np.allclose(cache.buf_score, 2 * before.astype(np.float64), rtol=1e-6)
+
+
+def test_buffer_mass_equal_keys_is_uniform_over_pools_and_block():
+    # identical keys everywhere (a constant row quantizes losslessly): every
+    # cached token gets 1/n of each head, so a block token gets H_q / n
+    B, Lyr, H, H_q, T, nb = 1, 1, 1, 4, 30, 5
+    cache = O.MixedCache(B, Lyr, H, 6, 5, 500_000)
+    k = np.full((B, Lyr, H, T, 128), 0.75, np.float16)
+    cache.prefill(k, k, [T], [O.select_mask(np.arange(T, dtype=np.float32), O.num_high(T, 500_000))])
+    kb = np.full((B, Lyr, H, nb, 128), 0.75, np.float16)
+    cache.append(kb, kb, np.zeros((B, nb), np.float32))
+    q = np.random.default_rng(3).standard_normal((B, Lyr, H_q, 128)).astype(np.float16)
+    cache.decode(q, score_layer=0)
+    assert np.allclose(cache.buf_score[0], H_q / (T + nb), rtol=1e-6)
+
+
 def test_decode_lossless_grid_cache_is_textbook_attention():
     # rows built on their own class's level grid quantize without loss, so the
     # mixed-cache decode must equal plain attention over the same values
