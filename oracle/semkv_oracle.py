@@ -168,11 +168,36 @@ def select_mask(score: np.ndarray, n_high: int) -> np.ndarray:
 #          (SemKV, Table 2 "integer-level scalar quantization"; Table 6: affine
 #          quantization stores two scalars per row)
 # ---------------------------------------------------------------------------
-def quantize_rows(xh: np.ndarray, L: int):
-    """Affine quantization of each row of D fp16 values to L levels.
+def fwht128(x: np.ndarray) -> np.ndarray:
+    """Unnormalised fast Walsh-Hadamard transform of each row of 128 values.
 
-    xh: float16 [..., D] -> (codes uint8 [..., D], mn float32 [...],
-    scale float32 [...], bad bool [...]).
+    SemKV, Table 2: the quantizer rotates each row with a Hadamard transform
+    before its min/max.  Stages h = 1, 2, 4, ..., 64 in that order; each
+    butterfly maps (a, b) at positions (j, j + h) to (a + b, a - b), one
+    rounding each in the dtype of x (float32 for the quantizer, float64 for
+    the reference decode).  H is symmetric and H H = 128 I, so the inverse is
+    the same transform divided by 128.
+    """
+    y = np.array(x, copy=True)
+    n = y.shape[-1]
+    if n != 128:
+        raise ValueError("rows must hold 128 values")
+    h = 1
+    while h < n:
+        v = y.reshape(y.shape[:-1] + (n // (2 * h), 2, h))
+        a = v[..., 0, :].copy()
+        b = v[..., 1, :].copy()
+        v[..., 0, :] = a + b
+        v[..., 1, :] = a - b
+        h *= 2
+    return y
+
+
+def quantize_rows(xh: np.ndarray, L: int):
+    """Affine quantization of each row of D values to L levels.
+
+    xh: float16 [..., D] (or float32 rows, e.g. rotated by fwht128) ->
+    (codes uint8 [..., D], mn float32 [...], scale float32 [...], bad bool [...]).
 
     Per row, in IEEE float32 with round-to-nearest-even:
       mn = min(x) + 0, mx = max(x) + 0   (adding +0 turns -0 into +0)
@@ -181,8 +206,8 @@ def quantize_rows(xh: np.ndarray, L: int):
     The two stored scalars are (mn, scale).  ``bad`` marks rows holding a
     non-finite value; their codes are unspecified.
     """
-    if xh.dtype != np.float16:
-        raise ValueError("rows must be float16")
+    if xh.dtype not in (np.float16, np.float32):
+        raise ValueError("rows must be float16 or float32")
     if xh.shape[0] == 0:
         shp = xh.shape[:-1]
         return (np.zeros(xh.shape, np.uint8), np.zeros(shp, np.float32), np.zeros(shp, np.float32),
@@ -250,13 +275,17 @@ class Pool:
     scale: np.ndarray   # float32 [n]
 
 
-def quantize_slab(x: np.ndarray, mask: np.ndarray, L_high: int, L_low: int):
+def quantize_slab(x: np.ndarray, mask: np.ndarray, L_high: int, L_low: int, rotate: bool = False):
     """Quantize the rows x [T][D] of one (sequence, layer, head) under one mask.
 
     Returns (high Pool, low Pool, bad rows).  Row j goes to the high pool when
     mask[j] == 1, else to the low pool; within a pool rows keep token order,
-    so a token's slot is the number of same-class tokens before it.
+    so a token's slot is the number of same-class tokens before it.  With
+    rotate, each fp16 row is first widened to float32 and rotated (fwht128),
+    and the rotated row is what is quantized and stored.
     """
+    if rotate:
+        x = fwht128(x.astype(np.float32))
     out = []
     bad_any = np.zeros(x.shape[0], dtype=bool)
     for cls, L in ((1, L_high), (0, L_low)):
@@ -292,8 +321,9 @@ class MixedCache:
     full, so a full block never stays in FP16.
     """
 
-    def __init__(self, B, Lyr, H, L_high, L_low, r_ppm, block=BLOCK, D=HEAD_DIM):
+    def __init__(self, B, Lyr, H, L_high, L_low, r_ppm, block=BLOCK, D=HEAD_DIM, rotate=False):
         self.B, self.Lyr, self.H, self.D = B, Lyr, H, D
+        self.rotate = rotate
         self.L_high, self.L_low, self.r_ppm, self.block = L_high, L_low, r_ppm, block
         self.slabs = [[[SlabCache() for _ in range(H)] for _ in range(Lyr)] for _ in range(B)]
         self.buf_k = np.zeros((B, Lyr, H, 0, D), dtype=np.float16)
@@ -309,7 +339,7 @@ class MixedCache:
             for h in range(self.H):
                 slab = self.slabs[b][l][h]
                 for x, hi_list, lo_list in ((k, slab.kh, slab.kl), (v, slab.vh, slab.vl)):
-                    ph, pl, bad = quantize_slab(x[l, h], mask, self.L_high, self.L_low)
+                    ph, pl, bad = quantize_slab(x[l, h], mask, self.L_high, self.L_low, self.rotate)
                     hi_list.append(ph)
                     lo_list.append(pl)
                     self.bad |= bool(bad.any())
@@ -374,14 +404,14 @@ class MixedCache:
                 keys, vals = [], []
                 for h in range(self.H):
                     kk, vv = [], []
-                    for which, L in (("kh", self.L_high), ("kl", self.L_low)):
-                        p = self.pools(b, l, h, which)
-                        if p.words.shape[0]:
-                            kk.append(dequantize(unpack_rows(p.words, L, D), p.mn, p.scale))
-                    for which, L in (("vh", self.L_high), ("vl", self.L_low)):
-                        p = self.pools(b, l, h, which)
-                        if p.words.shape[0]:
-                            vv.append(dequantize(unpack_rows(p.words, L, D), p.mn, p.scale))
+                    for dst, pair in ((kk, (("kh", self.L_high), ("kl", self.L_low))),
+                                      (vv, (("vh", self.L_high), ("vl", self.L_low)))):
+                        for which, L in pair:
+                            p = self.pools(b, l, h, which)
+                            if p.words.shape[0]:
+                                x = dequantize(unpack_rows(p.words, L, D), p.mn, p.scale)
+                                # stored rows are rotated: back to the token's own basis
+                                dst.append(fwht128(x) / 128.0 if self.rotate else x)
                     kk.append(self.buf_k[b, l, h].astype(np.float64))
                     vv.append(self.buf_v[b, l, h].astype(np.float64))
                     keys.append(np.concatenate(kk))

@@ -340,6 +340,46 @@ def test_generation_block_exact_counts():
     assert cache.buf_k.shape[3] == 0
 
 
+# ---------------------------------------------------------------- rotation (Hadamard, Table 2)
+def test_fwht128_matches_scipy_hadamard_matrix():
+    import scipy.linalg
+    Hm = scipy.linalg.hadamard(128).astype(np.float64)
+    rng = np.random.default_rng(31)
+    xi = rng.integers(-50, 51, (20, 128)).astype(np.float64)        # exact in any order
+    assert np.array_equal(O.fwht128(xi), xi @ Hm.T)
+    assert np.array_equal(O.fwht128(O.fwht128(xi)), 128.0 * xi)       # H H = 128 I
+    x = (rng.standard_normal((50, 128)) * rng.lognormal(0, 2, (50, 1))).astype(np.float32)
+    y = O.fwht128(x)
+    assert y.dtype == np.float32
+    exact = x.astype(np.float64) @ Hm.T
+    bound = 7 * 2.0 ** -24 * np.abs(x.astype(np.float64)).sum(axis=1, keepdims=True) * 2
+    assert np.all(np.abs(y - exact) <= bound)
+
+
+def test_rotated_quantizer_error_bound_and_outlier_spread():
+    # x_hat = H(dequant(q(Hx)))/128: each rotated value errs by at most
+    # scale/2 (+ fp32 slack), and the inverse transform averages 128 of them
+    rng = np.random.default_rng(32)
+    T = 400
+    x = rng.standard_normal((T, 128)).astype(np.float32)
+    x[:, [3, 50, 77, 120]] *= 10.0                                    # four outlier channels
+    xh = x.astype(np.float16)
+    for L in (5, 6):
+        mask = np.zeros(T, np.uint8) if L == 5 else np.ones(T, np.uint8)
+        ph, pl, bad = O.quantize_slab(xh, mask, 6, 5, rotate=True)
+        pool = ph if L == 6 else pl
+        rec = O.fwht128(O.dequantize(O.unpack_rows(pool.words, L), pool.mn, pool.scale)) / 128.0
+        err = np.abs(rec - xh.astype(np.float64))
+        assert not bad.any()
+        assert np.all(err <= pool.scale[:, None] * (0.5 + 2.0 ** -18) + 1e-5 * np.abs(pool.mn)[:, None] + 1e-6)
+        # outliers: the rotation spreads the four large channels over every dim,
+        # so the mean squared error is lower than without it
+        p2h, p2l, _ = O.quantize_slab(xh, mask, 6, 5, rotate=False)
+        p2 = p2h if L == 6 else p2l
+        rec2 = O.dequantize(O.unpack_rows(p2.words, L), p2.mn, p2.scale)
+        assert np.mean(err ** 2) < 0.5 * np.mean((rec2 - xh.astype(np.float64)) ** 2)
+
+
 # ---------------------------------------------------------------- a6 decode
 def test_decode_all_fp16_buffer_is_textbook_attention():
     rng = np.random.default_rng(12)
