@@ -73,6 +73,13 @@ typedef enum semkv_score_kind {
  * The FP16 block (Fig. 6): buf_k, buf_v fp16 [B][n_layers][H][block][128],
  * buf_score fp32 [B][block]; buf_len (HOST field) tokens of it are in use,
  * the same number for every sequence.
+ * rotate = 1 (SemKV, Table 2: the quantizer applies a Hadamard rotation):
+ * every K and V row x (fp16) is widened to fp32 and replaced by x' = H x, H
+ * the unnormalised 128-point Hadamard matrix computed by the fast transform
+ * with stages h = 1, 2, ..., 64 (one fp32 rounding per butterfly); x' is what
+ * is quantized and stored, (min, scale) are x''s.  Decode rotates q the same
+ * way and returns H o' / 128, so outputs are in the tokens' own basis.  The
+ * FP16 block is stored unrotated.  Needs H_q/H <= 4 (UNSUPPORTED otherwise).
  */
 typedef struct semkv_cache {
   int32_t B, n_layers, H, H_q, D;
@@ -81,6 +88,7 @@ typedef struct semkv_cache {
   int32_t cap_high, cap_low;     /* slots per (sequence, layer, head); multiples of 16 */
   int32_t block;                 /* FP16 block length (128)                          */
   int32_t buf_len;               /* host: tokens in the FP16 block, 0 <= buf_len < block */
+  int32_t rotate;                /* 0, or 1: Hadamard-rotated rows (Table 2), see below */
   uint32_t *k_high, *v_high, *k_low, *v_low;
   float *k_high_meta, *v_high_meta, *k_low_meta, *v_low_meta;
   int32_t *n_high, *n_low;       /* device [B] */

@@ -33,7 +33,7 @@ _i32, _i64, _u32, _sz, _f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, c
 class SemkvCache(ctypes.Structure):
     """Mirror of struct semkv_cache."""
     _fields_ = [(n, _i32) for n in ("B", "n_layers", "H", "H_q", "D", "L_high", "L_low", "r_ppm",
-                                     "cap_high", "cap_low", "block", "buf_len")] + \
+                                     "cap_high", "cap_low", "block", "buf_len", "rotate")] + \
                [(n, _p) for n in ("k_high", "v_high", "k_low", "v_low", "k_high_meta", "v_high_meta",
                                   "k_low_meta", "v_low_meta", "n_high", "n_low", "buf_k", "buf_v",
                                   "buf_score")]
@@ -145,7 +145,7 @@ class MixedCache:
     """
 
     def __init__(self, B, n_layers, H, H_q, L_high, L_low, r_ppm, cap_high, cap_low, block=128,
-                 device="cuda"):
+                 device="cuda", rotate=False):
         self.device = torch.device(device)
         cap_high = (int(cap_high) + 15) // 16 * 16
         cap_low = (int(cap_low) + 15) // 16 * 16
@@ -167,6 +167,7 @@ class MixedCache:
         self.buf_score = torch.zeros((B, block), dtype=torch.float32, device=d)
         self.status = torch.zeros(1, dtype=torch.int32, device=d)
         self.c = SemkvCache(B, n_layers, H, H_q, 128, L_high, L_low, r_ppm, cap_high, cap_low, block, 0,
+                            1 if rotate else 0,
                             *[t.data_ptr() for t in (self.k_high, self.v_high, self.k_low, self.v_low,
                                                      self.k_high_meta, self.v_high_meta, self.k_low_meta,
                                                      self.v_low_meta, self.n_high, self.n_low, self.buf_k,

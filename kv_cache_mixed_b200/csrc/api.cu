@@ -26,6 +26,8 @@ semkv_status check_cache(const semkv_cache *c) {
   if (c->r_ppm < 0 || c->r_ppm > 1000000) return SEMKV_ERR_INVALID_ARG;
   if (c->cap_high < 0 || c->cap_low < 0 || (c->cap_high % 16) || (c->cap_low % 16)) return SEMKV_ERR_INVALID_ARG;
   if (c->block < 1 || c->block > 128) return SEMKV_ERR_INVALID_ARG;
+  if (c->rotate != 0 && c->rotate != 1) return SEMKV_ERR_INVALID_ARG;
+  if (c->rotate && c->H_q / c->H > 4) return SEMKV_ERR_UNSUPPORTED;
   if (c->buf_len < 0 || c->buf_len >= c->block) return SEMKV_ERR_INVALID_ARG;
   const void *ptrs[] = {c->k_high, c->v_high, c->k_low, c->v_low, c->k_high_meta, c->v_high_meta,
                         c->k_low_meta, c->v_low_meta, c->n_high, c->n_low, c->buf_k, c->buf_v,
@@ -75,6 +77,7 @@ semkv_status quantize_rows(semkv_cache *c, const uint16_t *k, const uint16_t *v,
   q.cap_high = c->cap_high;
   q.cap_low = c->cap_low;
   q.L_high = c->L_high;
+  q.rotate = c->rotate;
   q.L_low = c->L_low;
   q.status = status;
   return cuda_status(launch_quantize(q, st));

@@ -204,6 +204,7 @@ struct DecParams {
   int NU, unit0, S;                 // units per slab, first unit of this launch, splits
   uint32_t *status;
   uint32_t Lrt;                     // the pool's level count (equals the template L)
+  int rot;                          // rows stored Hadamard-rotated (needs G <= 4)
 };
 
 constexpr int kMergeBytes = DEC_WARPS * DEC_GMAX * kD * 4 + DEC_WARPS * DEC_GMAX * 3 * 4;
@@ -219,7 +220,7 @@ constexpr int kLutBytes = 64 * 4;           // pair table, L*L <= 36 entries
 template <int L>
 constexpr int kQfragBytes = Geo<L>::KB * 32 * 8;   // q operand fragments, [kb][lane] x 2 words
 
-template <int L>
+template <int L, bool ROT>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 4)
 decode_pool_kernel(const DecParams p) {
   using Gm = Geo<L>;
@@ -253,10 +254,28 @@ decode_pool_kernel(const DecParams p) {
     qs[i] = __half2float(__ushort_as_half(hb));
   }
   __syncthreads();
+  if (ROT) {
+    // q' = H q (unnormalised 128-point Hadamard, fp32): q . k = q' . (H k) / 128
+    for (int h = 1; h < kD; h <<= 1) {
+      for (int i = threadIdx.x; i < G * (kD / 2); i += DEC_WARPS * 32) {
+        float *row = qs + (i / (kD / 2)) * kD;
+        const int bi = i % (kD / 2), j = (bi / h) * 2 * h + bi % h;
+        const float a = row[j], b = row[j + h];
+        row[j] = __fadd_rn(a, b);
+        row[j + h] = __fsub_rn(a, b);
+      }
+      __syncthreads();
+    }
+  }
 
   // ---- q fragments in slot order (kept in shared memory, one copy per CTA:
   // every warp uses the same fragments), and sum(q) * c2 for this lane's query r
+  // With rotated rows q' is not an f16 value: columns 0..3 carry its f16
+  // high part and columns 4..7 (G <= 4) its low part, q' - hi, so one MMA
+  // gives the logit to about 2^-22 relative.
   float qsum = 0.0f;
+  const bool qlo = ROT && r >= 4;
+  const int rq = ROT ? (r & 3) : r;
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) {
     uint32_t qv[2];
@@ -266,8 +285,9 @@ decode_pool_kernel(const DecParams p) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int d = slot_dim<L>(c, 4 * kb + 2 * hh + e);
-        v[e] = (r < G && d >= 0) ? qs[r * kD + d] : 0.0f;
-        qsum += v[e];
+        v[e] = (rq < G && d >= 0) ? qs[rq * kD + d] : 0.0f;
+        qsum += qlo ? 0.0f : v[e];
+        if (qlo) v[e] = __fsub_rn(v[e], __half2float(__float2half_rn(v[e])));
       }
       qv[hh] = pack_half2(v[0], v[1]);
     }
@@ -276,8 +296,9 @@ decode_pool_kernel(const DecParams p) {
   __syncthreads();
   qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
   qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
-  const float qsc = qsum * p.c2;
-  const float kscale = p.c2 * 16777216.0f;             // 2^24: codes are c * 2^-24
+  const float c2k = ROT ? p.c2 * (1.0f / 128.0f) : p.c2;     // rotated: q' . k' / 128
+  const float qsc = qsum * c2k;
+  const float kscale = c2k * 16777216.0f;              // 2^24: codes are c * 2^-24
   // This lane's two queries are the MMA columns 2c, 2c+1 of the logits.  With
   // G <= 4 the value MMA's columns 4..7 carry the low f16 part of P' for
   // queries 0..3, so lanes c >= 2 mirror the softmax of lane c-2 and one MMA
@@ -361,7 +382,8 @@ decode_pool_kernel(const DecParams p) {
       for (int i = 0; i < 4; ++i) {
         float sv = sa[i] + sb[i];
         const float mirror = __shfl_xor_sync(0xffffffffu, sv, 2);
-        if (pack_lo && c >= 2) sv = mirror;
+        if (ROT) sv = sv + mirror;                    // high + low part of q'
+        else if (pack_lo && c >= 2) sv = mirror;
         const int tt = (i < 2) ? r : 8 + r;
         const float2 mm = skm[tt];
         const float v = __fmaf_rn(sv, mm.y * kscale, mm.x * ((i & 1) ? qs1 : qs0));
@@ -596,6 +618,7 @@ __global__ void __launch_bounds__(128) decode_buffer_kernel(const BufParams p) {
 // layer, thread t < buf_len also writes the final softmax probability of
 // FP16 token t (same normalisation as the output) for the score accumulation.
 struct MergeAcc {
+  int rot;                     // pool partials are in the rotated basis: o = (H o' / 128 + o_buf) / l
   int score_li, block, buf_len;
   const float *logit;          // [B][H_q][block]
   float *prob;                 // [B][H_q][block]
@@ -604,21 +627,34 @@ struct MergeAcc {
 __global__ void __launch_bounds__(128) decode_merge_kernel(const float *__restrict__ part, int NU,
                                                            int G, int H, int nL, int H_q,
                                                            uint16_t *__restrict__ out, const MergeAcc acc) {
+  __shared__ float ot[kD];
   const int slab = blockIdx.x / G, qh = blockIdx.x % G, d = threadIdx.x;
   const int h = slab % H, li = (slab / H) % nL, b = slab / (H * nL);
   const float *pq = part + (int64_t)slab * NU * G * PART_STRIDE + qh * PART_STRIDE;
   float M = -INFINITY;
   for (int u = 0; u < NU; ++u) M = fmaxf(M, pq[(int64_t)u * G * PART_STRIDE]);
-  float o = 0.0f, l = 0.0f;
+  float o = 0.0f, l = 0.0f, ob = 0.0f;        // ob: the FP16 block's share (last unit)
   if (M != -INFINITY) {
     for (int u = 0; u < NU; ++u) {
       const float *pp = pq + (int64_t)u * G * PART_STRIDE;
       const float mu = pp[0];
       if (mu == -INFINITY) continue;
       const float a = ex2_approx(mu - M);
-      o += a * pp[4 + d];
+      if (acc.rot && u == NU - 1) ob = a * pp[4 + d];
+      else o += a * pp[4 + d];
       l += a * pp[1];
     }
+  }
+  if (acc.rot) {                               // uniform per CTA
+    ot[d] = o;
+    __syncthreads();
+    for (int hs = 1; hs < kD; hs <<= 1) {
+      const float a = ot[d & ~hs], bb = ot[d | hs];
+      __syncthreads();
+      ot[d] = (d & hs) ? __fsub_rn(a, bb) : __fadd_rn(a, bb);
+      __syncthreads();
+    }
+    o = __fmaf_rn(ot[d], 1.0f / 128.0f, ob);
   }
   const float res = l > 0.0f ? o / l : 0.0f;
   out[(((int64_t)b * nL + li) * H_q + h * G + qh) * kD + d] = __half_as_ushort(__float2half_rn(res));
@@ -645,42 +681,43 @@ static int pool_smem_bytes(int G) {
   return kQOff<L> + kLutBytes + kQfragBytes<L> + G * kD * 4;
 }
 
-template <int L>
+template <int L, bool ROT>
 static cudaError_t launch_pool(const DecParams &p, int grid, cudaStream_t st) {
   const int smem = pool_smem_bytes<L>(p.G);
-  static int attr_set = 0;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_pool_kernel<L>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         pool_smem_bytes<L>(DEC_GMAX));
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(decode_pool_kernel<L>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    attr_set = 1;
-  }
-  decode_pool_kernel<L><<<grid, DEC_WARPS * 32, smem, st>>>(p);
+  cudaError_t e = cudaFuncSetAttribute(decode_pool_kernel<L, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       pool_smem_bytes<L>(DEC_GMAX));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(decode_pool_kernel<L, ROT>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
+  decode_pool_kernel<L, ROT><<<grid, DEC_WARPS * 32, smem, st>>>(p);
   return cudaGetLastError();
 }
 
+template <bool ROT>
 static cudaError_t launch_pool_rt(int L, const DecParams &p, int grid, cudaStream_t st) {
   switch (L) {
-    case 2: return launch_pool<2>(p, grid, st);
-    case 3: return launch_pool<3>(p, grid, st);
-    case 4: return launch_pool<4>(p, grid, st);
-    case 5: return launch_pool<5>(p, grid, st);
-    case 6: return launch_pool<6>(p, grid, st);
-    case 7: return launch_pool<7>(p, grid, st);
-    case 8: return launch_pool<8>(p, grid, st);
-    case 9: return launch_pool<9>(p, grid, st);
-    case 10: return launch_pool<10>(p, grid, st);
-    case 11: return launch_pool<11>(p, grid, st);
-    case 12: return launch_pool<12>(p, grid, st);
-    case 13: return launch_pool<13>(p, grid, st);
-    case 14: return launch_pool<14>(p, grid, st);
-    case 15: return launch_pool<15>(p, grid, st);
-    case 16: return launch_pool<16>(p, grid, st);
+    case 2: return launch_pool<2, ROT>(p, grid, st);
+    case 3: return launch_pool<3, ROT>(p, grid, st);
+    case 4: return launch_pool<4, ROT>(p, grid, st);
+    case 5: return launch_pool<5, ROT>(p, grid, st);
+    case 6: return launch_pool<6, ROT>(p, grid, st);
+    case 7: return launch_pool<7, ROT>(p, grid, st);
+    case 8: return launch_pool<8, ROT>(p, grid, st);
+    case 9: return launch_pool<9, ROT>(p, grid, st);
+    case 10: return launch_pool<10, ROT>(p, grid, st);
+    case 11: return launch_pool<11, ROT>(p, grid, st);
+    case 12: return launch_pool<12, ROT>(p, grid, st);
+    case 13: return launch_pool<13, ROT>(p, grid, st);
+    case 14: return launch_pool<14, ROT>(p, grid, st);
+    case 15: return launch_pool<15, ROT>(p, grid, st);
+    case 16: return launch_pool<16, ROT>(p, grid, st);
     default: return cudaErrorInvalidValue;
   }
+}
+
+static cudaError_t launch_pool_any(int L, const DecParams &p, int grid, cudaStream_t st) {
+  return p.rot ? launch_pool_rt<true>(L, p, grid, st) : launch_pool_rt<false>(L, p, grid, st);
 }
 
 // splits per slab for a pool of capacity cap (host knows only capacities)
@@ -731,14 +768,15 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int sc
   p.km = reinterpret_cast<const float2 *>(c.k_high_meta);
   p.vm = reinterpret_cast<const float2 *>(c.v_high_meta);
   p.count = c.n_high; p.cap = c.cap_high; p.unit0 = 0; p.S = Sh; p.Lrt = (uint32_t)c.L_high;
-  e = launch_pool_rt(c.L_high, p, slabs * Sh, st);
+  p.rot = c.rotate;
+  e = launch_pool_any(c.L_high, p, slabs * Sh, st);
   if (e != cudaSuccess) return e;
   // low pool
   p.kw = c.k_low; p.vw = c.v_low;
   p.km = reinterpret_cast<const float2 *>(c.k_low_meta);
   p.vm = reinterpret_cast<const float2 *>(c.v_low_meta);
   p.count = c.n_low; p.cap = c.cap_low; p.unit0 = Sh; p.S = Sl; p.Lrt = (uint32_t)c.L_low;
-  e = launch_pool_rt(c.L_low, p, slabs * Sl, st);
+  e = launch_pool_any(c.L_low, p, slabs * Sl, st);
   if (e != cudaSuccess) return e;
   // FP16 block
   BufParams bp;
@@ -758,6 +796,7 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int sc
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   MergeAcc ma;
+  ma.rot = c.rotate;
   ma.score_li = score_li;
   ma.block = c.block;
   ma.buf_len = c.buf_len;

@@ -27,6 +27,7 @@ struct QuantLaunch {
   uint32_t *k_high, *v_high, *k_low, *v_low;
   float *k_high_meta, *v_high_meta, *k_low_meta, *v_low_meta;
   int cap_high, cap_low, L_high, L_low;
+  int rotate;                       // 1: Hadamard-rotate each row before quantizing
   uint32_t *status;
 };
 cudaError_t launch_quantize(const QuantLaunch &q, cudaStream_t st);

@@ -22,14 +22,14 @@ def to_np(t):
     return t.detach().cpu().numpy()
 
 
-def new_cache(B, Lyr, H, H_q, L_high, L_low, r_ppm, T_cap, block=128, gen=0):
+def new_cache(B, Lyr, H, H_q, L_high, L_low, r_ppm, T_cap, block=128, gen=0, rotate=False):
     kv = kv_mod()
     cap_h = O.num_high(T_cap, r_ppm) + O.num_high(block, r_ppm) * (gen // block + 2) + 16
     cap_l = T_cap + block * (gen // block + 2) + 16
-    return kv.MixedCache(B, Lyr, H, H_q, L_high, L_low, r_ppm, cap_h, cap_l, block=block)
+    return kv.MixedCache(B, Lyr, H, H_q, L_high, L_low, r_ppm, cap_h, cap_l, block=block, rotate=rotate)
 
 
-def compare_pools(cache, k, v, masks, seq_len, L_high, L_low, layers=None, heads=None):
+def compare_pools(cache, k, v, masks, seq_len, L_high, L_low, layers=None, heads=None, rotate=False):
     """Bit-exact comparison of every pool row of the given (layer, head) slabs."""
     B, Lyr, H = k.shape[0], k.shape[1], k.shape[2]
     layers = range(Lyr) if layers is None else layers
@@ -46,7 +46,7 @@ def compare_pools(cache, k, v, masks, seq_len, L_high, L_low, layers=None, heads
                         (k, (cache.k_high, cache.k_low, cache.k_high_meta, cache.k_low_meta)),
                         (v, (cache.v_high, cache.v_low, cache.v_high_meta, cache.v_low_meta))):
                     xs = to_np(x[b, l, h, :T]) if isinstance(x, torch.Tensor) else x[b, l, h, :T]
-                    ph, pl, _ = O.quantize_slab(xs, m, L_high, L_low)
+                    ph, pl, _ = O.quantize_slab(xs, m, L_high, L_low, rotate)
                     for pool, words, meta, n in ((ph, ph_w, ph_m, n_high[b]), (pl, pl_w, pl_m, n_low[b])):
                         gw = to_np(words[b, l, h, :n]).view(np.uint32)
                         gm = to_np(meta[b, l, h, :n])

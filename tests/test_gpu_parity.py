@@ -31,12 +31,12 @@ def _oracle_masks(score, seq_len, r_ppm):
     return [O.select_mask(s[b, :int(seq_len[b])], O.num_high(int(seq_len[b]), r_ppm)) for b in range(s.shape[0])]
 
 
-def _prefill(k, v, score, seq_len_t, L_high, L_low, r_ppm, H_q, block=128, gen=0):
+def _prefill(k, v, score, seq_len_t, L_high, L_low, r_ppm, H_q, block=128, gen=0, rotate=False):
     kv = kv_mod()
     B, Lyr, H, T = k.shape[:4]
     mask = torch.zeros((B, T), dtype=torch.uint8, device=DEV)
     kv.semkv_select(score, seq_len_t, r_ppm, mask)
-    cache = new_cache(B, Lyr, H, H_q, L_high, L_low, r_ppm, T, block=block, gen=gen)
+    cache = new_cache(B, Lyr, H, H_q, L_high, L_low, r_ppm, T, block=block, gen=gen, rotate=rotate)
     kv.semkv_quantize(cache, k, v, seq_len_t, mask)
     return cache, mask
 
@@ -387,8 +387,8 @@ def test_generation_block_exact(block, chunk):
     check_attention(to_np(out), ref.decode(q))
 
 
-@pytest.mark.parametrize("block", [16, 128])
-def test_generation_attention_mass_accumulation(block):
+@pytest.mark.parametrize("block,rotate", [(16, False), (128, False), (16, True)])
+def test_generation_attention_mass_accumulation(block, rotate):
     """Scores of generated tokens from the attention they receive at the scoring
     layer: buf_score matches the oracle within the score tolerance after every
     step, and each block is ranked on the GPU's accumulated scores (the oracle
@@ -407,8 +407,8 @@ def test_generation_attention_mass_accumulation(block):
     score_layer = Lyr - 1
     cache, _ = _prefill(torch.from_numpy(k).to(DEV), torch.from_numpy(v).to(DEV), torch.from_numpy(sc).to(DEV),
                         torch.tensor(lens, dtype=torch.int32, device=DEV), L_high, L_low, r_ppm, H_q,
-                        block=block, gen=steps)
-    ref = O.MixedCache(B, Lyr, H, L_high, L_low, r_ppm, block=block)
+                        block=block, gen=steps, rotate=rotate)
+    ref = O.MixedCache(B, Lyr, H, L_high, L_low, r_ppm, block=block, rotate=rotate)
     ref.prefill(k, v, lens, _oracle_masks(torch.from_numpy(sc), lens, r_ppm))
     zeros = np.zeros((B, 1), np.float32)
     for step in range(steps):
@@ -463,6 +463,50 @@ def test_decode_attn_acc_is_deterministic_and_matches_plain_decode():
     assert float(d1[0, 50:].abs().max()) == 0.0                       # only the 50 block tokens
     with pytest.raises(kv.SemkvError):
         kv.semkv_decode_attn_acc(cache, 0, 1, 1, q[:, :1].contiguous(), o2[:, :1].contiguous())
+
+
+# ----------------------------------------------------------------- Hadamard rotation (Table 2)
+@pytest.mark.parametrize("L_high,L_low,kdist", [(6, 5, "x10ch"), (6, 5, "lognormal"), (8, 6, "x10ch"),
+                                                (4, 4, "x10ch"), (16, 2, "lognormal")])
+def test_rotated_quantize_bit_exact_and_decode(L_high, L_low, kdist):
+    kv = kv_mod()
+    wl = synth.scaled(synth.TINY, B=2, Lyr=2, H=2, H_q=8, T=333, kdist=kdist)
+    k, v = synth.kv(wl, 300 + L_high, DEV)
+    score = synth.uniform_score(wl, L_low, DEV)
+    seq_len = torch.tensor([333, 201], dtype=torch.int32, device=DEV)
+    cache, mask = _prefill(k, v, score, seq_len, L_high, L_low, 500_000, wl.H_q, rotate=True)
+    masks = _oracle_masks(score, [333, 201], 500_000)
+    assert _status(cache) == 0
+    kn, vn = to_np(k), to_np(v)
+    compare_pools(cache, kn, vn, masks, [333, 201], L_high, L_low, rotate=True)
+    ref = O.MixedCache(2, 2, 2, L_high, L_low, 500_000, rotate=True)
+    ref.prefill(kn, vn, [333, 201], masks)
+    q = synth.decode_query(wl, 9, DEV)
+    out = torch.empty_like(q)
+    kv.semkv_decode_attn(cache, 0, 2, q, out)
+    check_attention(to_np(out), ref.decode(to_np(q)))
+
+
+def test_rotated_adversarial_rows_bit_exact():
+    kv = kv_mod()
+    rng = np.random.default_rng(404)
+    rows = _adversarial_rows(rng, 160)
+    x = rows.reshape(1, 1, 1, 160, 128)
+    sc = torch.from_numpy(rng.random((1, 160)).astype(np.float32)).to(DEV)
+    xt = torch.from_numpy(x).to(DEV)
+    cache, mask = _prefill(xt, xt, sc, torch.tensor([160], dtype=torch.int32, device=DEV), 6, 5, 500_000, 4,
+                           rotate=True)
+    masks = _oracle_masks(sc, [160], 500_000)
+    assert _status(cache) == 0
+    compare_pools(cache, x, x, masks, [160], 6, 5, rotate=True)
+
+
+def test_rotation_needs_at_most_four_query_heads_per_kv_head():
+    kv = kv_mod()
+    cache = new_cache(1, 1, 1, 8, 6, 5, 500_000, 64, rotate=True)
+    q = torch.zeros((1, 1, 8, 128), dtype=torch.float16, device=DEV)
+    with pytest.raises(kv.SemkvError):
+        kv.semkv_decode_attn(cache, 0, 1, q, torch.empty_like(q))
 
 
 def test_decode_layer_subset_and_empty_sequence():

@@ -51,16 +51,17 @@ def test_invalid_arguments_rejected_before_launch(kv):
     # a cache with D != 128, bad levels, unaligned pointers, bad capacities
     def cache(**kw):
         base = dict(B=1, n_layers=1, H=1, H_q=4, D=128, L_high=6, L_low=5, r_ppm=500_000, cap_high=16,
-                    cap_low=16, block=128, buf_len=0)
+                    cap_low=16, block=128, buf_len=0, rotate=0)
         base.update(kw)
         c = b.SemkvCache(*[base[k] for k in ("B", "n_layers", "H", "H_q", "D", "L_high", "L_low", "r_ppm",
-                                              "cap_high", "cap_low", "block", "buf_len")])
-        for f, _ in b.SemkvCache._fields_[12:]:
+                                              "cap_high", "cap_low", "block", "buf_len", "rotate")])
+        for f, _ in b.SemkvCache._fields_[13:]:
             setattr(c, f, 0x10000)
         return c
     for kw, want in [(dict(D=64), UNSUP), (dict(L_high=17), UNSUP), (dict(L_low=1), UNSUP),
                      (dict(H_q=3, H=2), INVALID), (dict(H_q=36, H=4), UNSUP), (dict(r_ppm=-1), INVALID),
-                     (dict(cap_high=17), INVALID), (dict(block=0), INVALID), (dict(buf_len=128), INVALID)]:
+                     (dict(cap_high=17), INVALID), (dict(block=0), INVALID), (dict(buf_len=128), INVALID),
+                     (dict(rotate=2), INVALID), (dict(rotate=1, H_q=8, H=1), UNSUP)]:
         c = cache(**kw)
         assert b._lib_decode(ctypes.byref(c), 0, 1, ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), 1.0,
                              ctypes.c_void_p(0x10000), 1 << 20, None, None) == want, kw
@@ -79,6 +80,11 @@ def test_invalid_arguments_rejected_before_launch(kv):
                          ctypes.c_void_p(0x10000), 1 << 20, None, None) == INVALID
     assert b._lib_decode(ctypes.byref(c), 0, 1, ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), -1.0,
                          ctypes.c_void_p(0x10000), 1 << 20, None, None) == INVALID
+    # decode with score accumulation: the scoring layer must be one of the decoded layers
+    assert b._lib_decode_acc(ctypes.byref(c), 0, 1, 1, ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), 1.0,
+                             ctypes.c_void_p(0x10000), 1 << 20, None, None) == INVALID
+    assert b._lib_decode_acc(ctypes.byref(c), 0, 1, -1, ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), 1.0,
+                             ctypes.c_void_p(0x10000), 1 << 20, None, None) == INVALID
     # append: negative n, unknown flag
     assert b._lib_append(ctypes.byref(c), None, None, None, -1, 0, ctypes.c_void_p(0x10000), 1 << 20,
                          None, None) == INVALID
