@@ -290,6 +290,49 @@ def run_ours(args, rank, world, dist):
     return res, (k, v, q_win, qdec, kn, vn, sn, seq_len, score, mask, out, cache, score_ws, fp16_in)
 
 
+def run_extensions(state, reps=5):
+    """Device times of the two options next to the headline path, on the same
+    workload: decode with attention-mass accumulation for the FP16 block at
+    the scoring layer, and the Hadamard-rotated cache (quantize and decode)."""
+    import torch
+
+    import kv_cache_mixed_b200 as kv
+    from inputs import synth
+    k, v, q_win, qdec, kn, vn, sn, seq_len, score, mask, out, cache, score_ws, fp16_in = state
+    wl = synth.LLAMA_PREFILL
+    B, Lyr, H, H_q, T = wl.B, wl.Lyr, wl.H, wl.H_q, wl.T
+    stream = torch.cuda.current_stream()
+
+    def timed(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for _ in range(reps):
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    acc_ms = timed(lambda: kv.semkv_decode_attn_acc(cache, 0, Lyr, Lyr - 1, qdec, out))
+    nh = kv.semkv_num_high(T, wl.r_ppm)
+    rc = kv.MixedCache(B, Lyr, H, H_q, wl.L_high, wl.L_low, wl.r_ppm, nh + 128, T - nh + 128, rotate=True)
+
+    def rq():
+        rc.n_high.zero_()
+        rc.n_low.zero_()
+        kv.semkv_quantize(rc, k, v, seq_len, mask)
+    rq_ms = timed(rq)
+    rd_ms = timed(lambda: kv.semkv_decode_attn(rc, 0, Lyr, qdec, out))
+    assert rc.status_flags() == 0 and cache.status_flags() == 0
+    return {"decode_acc_ms": round(acc_ms, 4),
+            "rotated": {"quantize_ms": round(rq_ms, 4), "decode_ms": round(rd_ms, 4),
+                        "quantize_gbs_fp16_in": round(fp16_in / (rq_ms * 1e-3) / 1e9, 1)}}
+
+
 def run_e2e(args, state, dist=None):
     """Same step through the C ABI with pinned HOST inputs: H2D copies of K, V,
     the query window, the decode query and the new token inside the timed
@@ -471,6 +514,7 @@ def main():
         return
     rank, world, dist = init_ranks("nccl")
     res, state = run_ours(args, rank, world, dist)
+    res["options"] = run_extensions(state)
     if not args.no_e2e:
         e2e = run_e2e(args, state, dist)
         if dist:

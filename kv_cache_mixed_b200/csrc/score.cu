@@ -419,7 +419,9 @@ template <int PASS>
 __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnParams p, int Np, int nchunk,
                                                                    float *head_part) {
   extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // 1024-byte alignment by an offset from the shared base, so that the compiler
+  // still sees shared-memory pointers (plain shared loads, not generic ones)
+  uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quarter = warp & 3, half = warp >> 2;
