@@ -49,6 +49,7 @@ def parse(argv=None):
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-options", action="store_true", help="skip the option timings (score accumulation, rotation)")
     ap.add_argument("--case", default=None, choices=["score", "select", "quantize", "decode"],
                     help="profiling case: run only this stage, on the prefill workload cut to --layers layers")
     ap.add_argument("--layers", type=int, default=4)
@@ -514,7 +515,8 @@ def main():
         return
     rank, world, dist = init_ranks("nccl")
     res, state = run_ours(args, rank, world, dist)
-    res["options"] = run_extensions(state)
+    if not args.no_options:
+        res["options"] = run_extensions(state)
     if not args.no_e2e:
         e2e = run_e2e(args, state, dist)
         if dist:
