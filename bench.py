@@ -225,19 +225,27 @@ def run_ours(args, rank, world, dist):
         torch.cuda.synchronize()
     # the step loop above synchronizes per step for the stage events; the
     # headline is also timed without those syncs below
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    t2, t3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # the clock sampler (one reading per 200 ms) starts with an untimed soak of
+    # about 0.4 s of steps, so that it holds several readings under load next
+    # to the short timed loop
+    step_ms = max(statistics.median([sum(times[n][i] for n in times) for i in range(len(times["score"]))]), 1e-3)
+    soak = int(400.0 / step_ms) + 1
     with Clocks(torch.cuda.current_device()) as clk2:
+        for _ in range(soak):
+            step(False)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t2, t3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t2.record(stream)
         for _ in range(args.steps):
             step(False)
         t3.record(stream)
         torch.cuda.synchronize()
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
     ms = t2.elapsed_time(t3) / args.steps
     assert cache.status_flags() == 0, "device status flags set"
     ms = max_over_ranks(ms, dist, dev)

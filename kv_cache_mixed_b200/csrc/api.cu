@@ -25,6 +25,7 @@ semkv_status check_cache(const semkv_cache *c) {
   if (c->L_high < 2 || c->L_high > kMaxL || c->L_low < 2 || c->L_low > kMaxL) return SEMKV_ERR_UNSUPPORTED;
   if (c->r_ppm < 0 || c->r_ppm > 1000000) return SEMKV_ERR_INVALID_ARG;
   if (c->cap_high < 0 || c->cap_low < 0 || (c->cap_high % 16) || (c->cap_low % 16)) return SEMKV_ERR_INVALID_ARG;
+  if (c->cap_high >= (1 << 30) || c->cap_low >= (1 << 30)) return SEMKV_ERR_INVALID_ARG;   // pool positions fit 30 bits
   if (c->block < 1 || c->block > 128) return SEMKV_ERR_INVALID_ARG;
   if (c->rotate != 0 && c->rotate != 1) return SEMKV_ERR_INVALID_ARG;
   if (c->rotate && c->H_q / c->H > 4) return SEMKV_ERR_UNSUPPORTED;
@@ -49,7 +50,8 @@ semkv_status quantize_rows(semkv_cache *c, const uint16_t *k, const uint16_t *v,
                            int64_t mask_bstride, void *ws, uint32_t *status, cudaStream_t st) {
   int32_t *slot = reinterpret_cast<int32_t *>(ws);
   int32_t *cnt = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(ws) + up256((size_t)c->B * T_stride * 4));
-  cudaError_t e = launch_slot_scan(mask, mask_bstride, seq_len, len_const, c->B, T_stride, slot, cnt, status, st);
+  cudaError_t e = launch_slot_scan(mask, mask_bstride, seq_len, len_const, c->B, T_stride, c->n_high, c->n_low,
+                                   slot, cnt, status, st);
   if (e != cudaSuccess) return SEMKV_ERR_CUDA;
   QuantLaunch q;
   q.k = k;
