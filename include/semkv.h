@@ -24,8 +24,9 @@
  *   - Conditions only the GPU can see (a non-finite input, a pool that would
  *     overflow, a length beyond T_max) are OR-ed as SEMKV_FLAG_* bits into the
  *     caller's device word `status` (may be NULL for calls that take none);
- *     the caller reads it after synchronizing.  Kernels never trap and never
- *     spin-wait.
+ *     the caller reads it after synchronizing.  Kernels never trap, and every
+ *     wait for an asynchronous copy or tensor-core result is bounded (a wait
+ *     that gives up sets SEMKV_FLAG_TIMEOUT).
  *   - D (head_dim) must be 128; level counts L must be in [2, 16].
  */
 #ifndef SEMKV_H
@@ -41,7 +42,7 @@ extern "C" {
 typedef enum semkv_status {
   SEMKV_OK = 0,
   SEMKV_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape    */
-  SEMKV_ERR_UNSUPPORTED = 2,   /* D != 128, L outside [2,16], H_q/H > 8          */
+  SEMKV_ERR_UNSUPPORTED = 2,   /* D != 128, L outside [2,16], H_q/H > 8 (> 4 with rotate) */
   SEMKV_ERR_WORKSPACE = 3,     /* workspace smaller than the *_workspace_size    */
   SEMKV_ERR_CAPACITY = 4,      /* an append would overflow the FP16 block        */
   SEMKV_ERR_CUDA = 5           /* a launch failed (cudaGetLastError)             */
@@ -171,7 +172,8 @@ size_t semkv_quantize_workspace_size(int32_t B, int32_t T_max);
  * Quantize every row of K and V [B][n_layers][H][T_max][D] (fp16) with tokens
  * j < seq_len[b], row class from mask[b][j] (1 = high), and append the rows to
  * the pools after the slots already in use (n_high[b], n_low[b]), which are
- * then advanced.  Per row, in IEEE fp32 round-to-nearest-even:
+ * then advanced.  With c->rotate the row x below is the rotated row H x (fp32,
+ * see the cache struct).  Per row, in IEEE fp32 round-to-nearest-even:
  *   mn = min(x)+0, mx = max(x)+0, scale = (mx-mn)/(L-1),
  *   code = scale == 0 ? 0 : clamp(rint((x-mn)/scale), 0, L-1)      (exact division)
  *   word w = sum_j code[w*n+j] * L^j, n = semkv_digits_per_word(L)  (little-endian digits)
