@@ -397,8 +397,8 @@ __global__ void __launch_bounds__(AM_WARPS * 32, 1) attn_colsum_kernel(const Att
 //           its chunk, and writes one partial per (row, chunk);
 //   pass 2: D[keys][rows] = K . Q_g^T  (M=128 keys, N=Np): each thread owns one
 //           key (warps w and w+4 split the rows) and sums exp2(s*c1 - M'_r),
-//           M'_r = M_r + log2(Z_r); one partial per (head, key), summed over
-//           heads in order by attn_headsum_kernel.
+//           M'_r = M_r + log2(Z_r); one partial per (head, row half, key),
+//           summed in order by attn_headsum_kernel.
 constexpr int UA_THREADS = 256;
 constexpr int UA_KEYS = 128;
 constexpr int UA_MAXN = 256;
@@ -408,8 +408,7 @@ constexpr int UA_KBYTES = UA_KEYS * 256;
 constexpr int UA_OFF_Q = 0;
 constexpr int UA_OFF_K = UA_QBYTES;
 constexpr int UA_OFF_M = UA_OFF_K + UA_NST * UA_KBYTES;          // float [256] M'_r (pass 2)
-constexpr int UA_OFF_X = UA_OFF_M + UA_MAXN * 4;                  // float [2][128] half-sum exchange
-constexpr int UA_OFF_BAR = UA_OFF_X + 2 * 128 * 4;                // u64 [2]
+constexpr int UA_OFF_BAR = UA_OFF_M + UA_MAXN * 4;                // u64 [2]
 constexpr int UA_OFF_SLOT = UA_OFF_BAR + 16;
 constexpr int UA_SMEM = UA_OFF_SLOT + 16 + 1024;
 constexpr int kUmmaWait = 1 << 22;
@@ -431,7 +430,6 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   const int tb = (int)((int64_t)ntile * chunk / nchunk), te = (int)((int64_t)ntile * (chunk + 1) / nchunk);
 
   float *Ms = reinterpret_cast<float *>(smem + UA_OFF_M);
-  float *xch = reinterpret_cast<float *>(smem + UA_OFF_X);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + UA_OFF_BAR);
   uint32_t *slot = reinterpret_cast<uint32_t *>(smem + UA_OFF_SLOT);
   const uint32_t sbase = smem_u32(smem);
@@ -595,14 +593,10 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
           }
         }
         const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-        // the two column halves of this key: warp w+4 hands its sum to warp w
-        float *xb = xch + ab * 128;                // by accumulator: the next write to it follows a barrier
-        if (half == 1) xb[quarter * 32 + lane] = acc;
-        tc_fence_before();
-        __syncthreads();
-        if (half == 0 && key < p.T_max)
-          head_part[((int64_t)b * p.H + g) * p.T_max + key] = key < len ? acc + xb[quarter * 32 + lane] : 0.0f;
-        continue;
+        // one partial per (KV head, column half, key): no exchange between the
+        // two warps of a key, the head-sum kernel adds the halves in order
+        if (key < p.T_max)
+          head_part[(((int64_t)b * p.H + g) * 2 + half) * p.T_max + key] = key < len ? acc : 0.0f;
       }
       tc_fence_before();
     }
@@ -623,7 +617,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
-// score[b][j] = sum over KV heads, in order, of the per-head column partials
+// score[b][j] = sum over KV heads and row halves, in order, of the column partials
 __global__ void attn_headsum_kernel(const AttnParams p, const float *__restrict__ head_part) {
   const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= (int64_t)p.B * p.T_max) return;
@@ -636,7 +630,7 @@ __global__ void attn_headsum_kernel(const AttnParams p, const float *__restrict_
   }
   float s = 0.0f;
   if (j < len)
-    for (int g = 0; g < p.H; ++g) s += head_part[((int64_t)b * p.H + g) * p.T_max + j];
+    for (int g = 0; g < 2 * p.H; ++g) s += head_part[((int64_t)b * 2 * p.H + g) * p.T_max + j];
   p.score[idx] = s;
 }
 
@@ -645,7 +639,7 @@ size_t attn_mass_ws_bytes(int B, int T_max, int H, int H_q, int w) {
   const int ntile = (T_max + AM_TILE - 1) / AM_TILE;
   const int nchunk = ntile < 64 ? ntile : 64;
   const size_t parts = (size_t)(rows * nchunk * sizeof(float2) + rows * sizeof(float2) + 256);
-  return (parts + 255) / 256 * 256 + (size_t)B * H * T_max * sizeof(float) + 256;
+  return (parts + 255) / 256 * 256 + (size_t)B * H * 2 * T_max * sizeof(float) + 256;
 }
 
 cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const uint16_t *q_win,
