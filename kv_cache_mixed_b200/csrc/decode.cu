@@ -726,8 +726,11 @@ static int pool_splits(const semkv_cache &c, int n_layers, int cap) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int64_t slabs = (int64_t)c.B * n_layers * c.H;
-  const int64_t target = (int64_t)sms * 12;           // ~4 waves of 3 CTAs per SM
-  int64_t S = (target + slabs - 1) / slabs;
+  // about 1.75 waves of the 4 resident CTAs per SM, rounded to the nearest
+  // split count: on the 32-layer prefill cache (256 slabs) 4 splits took
+  // 0.584 ms against 0.666 (2), 0.675 (3), 0.616 (5), 0.627 (7), 0.614 (10)
+  const int64_t target = (int64_t)sms * 7;
+  int64_t S = (target + slabs / 2) / slabs;
   const int64_t max_by_tiles = (cap / 16 + 15) / 16;  // keep >= 16 tiles (4 per warp) per unit
   if (S > max_by_tiles) S = max_by_tiles;
   if (S < 1) S = 1;
