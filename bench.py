@@ -437,7 +437,8 @@ def oracle_threads():
 
 
 def cpu_baseline_json():
-    per_step, desc = oracle_step_sample()
+    # 7 of 32 layers: about 10 s of host work on the GPU machine
+    per_step, desc = oracle_step_sample(7)
     fp16_in = 2 * 32 * 8 * 32768 * 128 * 2
     return {"value": round(fp16_in / per_step / 1e9, 4), "unit": "GB/s", "cores": oracle_threads(),
             "kind": "oracle", "sample": desc}
