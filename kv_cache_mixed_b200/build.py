@@ -2,7 +2,7 @@
 
     python kv_cache_mixed_b200/build.py [--force]
 
-(Run it as a file: importing the package loads the library this builds.)
+(Run it as a file: importing the package loads the library it compiles.)
 
 Objects go to kv_cache_mixed_b200/_build/, the library to
 kv_cache_mixed_b200/libsemkv.so.  A source newer than the library triggers a

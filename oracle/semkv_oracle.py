@@ -499,5 +499,5 @@ def pages_effective_bits(levels_and_fracs, meta_scalars: int, D: int = HEAD_DIM)
 
 
 def layout_bytes_per_row(L: int, D: int = HEAD_DIM) -> int:
-    """Bytes of one row in this build's layout: 32-bit mixed-radix words + fp32 (mn, scale)."""
+    """Bytes of one row in the library's layout: 32-bit mixed-radix words + fp32 (mn, scale)."""
     return 4 * words_per_row(L, D) + 8
