@@ -15,15 +15,18 @@
 // parts of k digits with L^k small enough that, with F = v * ceil(2^32/L^k),
 // each step t = F * L yields the next digit (most significant first) in the
 // high 32 bits and the next F in the low 32 bits.  The part sizes below were
-// checked exhaustively against repeated division for every part value.
+// checked exhaustively against repeated division for every part value.  For
+// L <= 6 one step by L^2 yields two digits, turned into the f16x2 operand by a
+// small shared-memory table.
 //
-// Work split: one pool class per launch (template on its L); CTA = 4 warps on
-// a contiguous range of 16-token tiles of one (sequence, layer, KV head); each
-// warp streams its tiles through a cp.async ring in shared memory; online
-// softmax in the log2 domain; the 4 warps merge in shared memory and the CTA
-// writes one partial (m, l, o[128]) per query head.  The FP16 block gets its
-// own small kernel and a last kernel merges all partials of a (sequence,
-// layer, KV head) into the output.
+// Work split: one pool class per launch (template on its L, and on whether
+// the rows are Hadamard-rotated); CTA = 4 warps on a contiguous range of
+// 16-token tiles of one (sequence, layer, KV head); each warp streams its
+// tiles through a ring of bulk asynchronous copies (cp.async.bulk completing
+// on mbarriers, bounded waits); online softmax in the log2 domain; the 4
+// warps merge in shared memory and the CTA writes one partial (m, l, o[128])
+// per query head.  The FP16 block gets its own small kernel and a last kernel
+// merges all partials of a (sequence, layer, KV head) into the output.
 //
 // MMA shapes per 16-token tile: the logits put the 16 tokens on the MMA rows
 // and the query heads on the 8 columns (one m16n8k16 per 16 head-dim slots);
