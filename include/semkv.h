@@ -113,6 +113,19 @@ int32_t semkv_words_per_row(int32_t L, int32_t D);
 /* Library build identification string (static storage). */
 const char *semkv_version(void);
 
+/*
+ * Testing aid for the bounded waits (no counterpart on the pages).  Sets how
+ * many times the FIRST wait of every warp's bulk-copy ring polls its mbarrier
+ * in semkv_quantize and semkv_decode_attn launches enqueued after this call
+ * (process-wide, not thread-safe).  polls < 0 restores each kernel's own bound
+ * (the default).  polls = 0 makes that wait give up at once, so the launch
+ * takes its timeout path: SEMKV_FLAG_TIMEOUT is set, the outputs of the warps
+ * concerned are unspecified, and every copy already issued is still waited
+ * for, with the default bound, before the warp exits.  No other wait is
+ * affected.  Not for production use.
+ */
+void semkv_set_first_copy_wait_polls(int32_t polls);
+
 /* ---- a1: importance score (Fig. 2) ---------------------------------------- */
 
 /* Workspace bytes semkv_score needs for these sizes (0 for KEY_L2). */
@@ -205,7 +218,11 @@ semkv_status semkv_quantize(semkv_cache *c, const uint16_t *k, const uint16_t *v
  *   - every call on a device uses the same array, which keeps the last call's
  *     contents: calls whose work overlaps on the GPU (other streams, other
  *     threads) race, so serialize them;
- *   - it calls no allocator: no cudaMalloc, cudaFree or allocating library.
+ *   - it calls no allocator: no cudaMalloc, cudaFree or allocating library;
+ *   - the looked-up address is kept for the life of the process: after
+ *     cudaDeviceReset (or anything else that tears down the device's primary
+ *     context) it is stale, so do not call this entry point on that device
+ *     again in the same process.
  * Arguments, results, flags and errors are otherwise those of semkv_quantize.
  */
 #define SEMKV_NOALLOC_SCRATCH_BYTES (4u << 20)

@@ -50,6 +50,7 @@ _lib_num_high = _sig("semkv_num_high", _i64, [_i64, _i32])
 _lib_digits = _sig("semkv_digits_per_word", _i32, [_i32])
 _lib_words = _sig("semkv_words_per_row", _i32, [_i32, _i32])
 _lib_version = _sig("semkv_version", ctypes.c_char_p, [])
+_lib_set_wait0 = _sig("semkv_set_first_copy_wait_polls", None, [_i32])
 _lib_score_ws = _sig("semkv_score_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32, _i32])
 _lib_score = _sig("semkv_score", _i32, [_i32, _p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _i32,
                                         _p, _p, _sz, _p, _p])
@@ -69,6 +70,7 @@ _lib_decode_acc = _sig("semkv_decode_attn_acc", _i32, [ctypes.POINTER(SemkvCache
                                                       _p, _sz, _p, _p])
 
 EXPORTED = ["semkv_num_high", "semkv_digits_per_word", "semkv_words_per_row", "semkv_version",
+            "semkv_set_first_copy_wait_polls",
             "semkv_score_workspace_size", "semkv_score", "semkv_select_workspace_size", "semkv_select",
             "semkv_quantize_workspace_size", "semkv_quantize", "semkv_quantize_noalloc",
             "semkv_append_workspace_size",
@@ -112,6 +114,11 @@ def semkv_words_per_row(L: int, D: int = 128) -> int:
 
 def semkv_version() -> str:
     return _lib_version().decode()
+
+
+def semkv_set_first_copy_wait_polls(polls: int) -> None:
+    """Testing aid: poll bound of the first copy wait of later quantize/decode launches (< 0: default)."""
+    _lib_set_wait0(int(polls))
 
 
 # ------------------------------------------------------------------ a1 score

@@ -10,6 +10,11 @@
 
 using namespace semkv;
 
+namespace semkv {
+static int g_first_wait_polls = -1;     // < 0: each kernel's own bound
+int first_wait_polls(int dflt) { return g_first_wait_polls < 0 ? dflt : g_first_wait_polls; }
+}  // namespace semkv
+
 namespace {
 
 inline bool al16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -125,7 +130,9 @@ int32_t semkv_words_per_row(int32_t L, int32_t D) {
   return (D + n - 1) / n;
 }
 
-const char *semkv_version(void) { return "semkv-b200 0.1 (sm_100a)"; }
+const char *semkv_version(void) { return "semkv-b200 0.2 (sm_100a)"; }
+
+void semkv_set_first_copy_wait_polls(int32_t polls) { g_first_wait_polls = polls < 0 ? -1 : polls; }
 
 size_t semkv_score_workspace_size(int32_t kind, int32_t B, int32_t T_max, int32_t H, int32_t H_q,
                                   int32_t w) {

@@ -208,6 +208,7 @@ struct DecParams {
   uint32_t *status;
   uint32_t Lrt;                     // the pool's level count (equals the template L)
   int rot;                          // rows stored Hadamard-rotated (needs G <= 4)
+  int wait0;                        // polls of each warp's first copy wait (testing aid)
 };
 
 constexpr int kMergeBytes = DEC_WARPS * DEC_GMAX * kD * 4 + DEC_WARPS * DEC_GMAX * 3 * 4;
@@ -355,7 +356,7 @@ decode_pool_kernel(const DecParams p) {
   for (; tile < te; tile += DEC_WARPS) {
     issue(next, (slotix + DEC_NST - 1) % DEC_NST);
     next += DEC_WARPS;
-    if (!mbar_wait(&bars[slotix], (parity >> slotix) & 1u, kWaitLimit)) {
+    if (!mbar_wait(&bars[slotix], (parity >> slotix) & 1u, tile == tb + warp ? p.wait0 : kWaitLimit)) {
       lost = true;
       break;
     }
@@ -563,54 +564,81 @@ struct BufParams {
   float *logit;                // [B][H_q][block] log2-domain logits of the FP16 tokens
 };
 
+// Logits: one warp per token, lane l holding dims 4l..4l+3, so each warp load
+// is one whole 256-byte row; the G partial dots are reduced by xor shuffles.
+// Values: thread = head dim, each V row read once (coalesced) for all G heads.
 __global__ void __launch_bounds__(128) decode_buffer_kernel(const BufParams p) {
   __shared__ float qs[DEC_GMAX][kD];
-  __shared__ float sc[DEC_GMAX][128];
+  __shared__ float pr[DEC_GMAX][128];    // logits (log2 domain), then exp2(logit - max)
   __shared__ float red[DEC_GMAX][2];
   const int slab = blockIdx.x;
   const int h = slab % p.H, li = (slab / p.H) % p.nL, b = slab / (p.H * p.nL);
   const int64_t pslab = ((int64_t)b * p.Lyr + p.layer0 + li) * p.H + h;
-  const int G = p.G, n = p.buf_len, tid = threadIdx.x;
+  const int G = p.G, n = p.buf_len, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   for (int i = tid; i < G * kD; i += 128)
     qs[i / kD][i % kD] = __half2float(__ushort_as_half(
         p.q[(((int64_t)b * p.nL + li) * p.H_q + h * G + i / kD) * kD + i % kD]));
   __syncthreads();
   const uint16_t *kb = p.bk + pslab * p.block * kD;
   const uint16_t *vb = p.bv + pslab * p.block * kD;
-  if (tid < n) {
-    for (int qh = 0; qh < G; ++qh) {
-      float acc = 0.0f;
-      for (int d = 0; d < kD; ++d) acc = fmaf(qs[qh][d], __half2float(__ushort_as_half(kb[(int64_t)tid * kD + d])), acc);
-      sc[qh][tid] = acc * p.c2;
-      if (li == p.score_li) p.logit[((int64_t)b * p.H_q + h * G + qh) * p.block + tid] = acc * p.c2;
-    }
-  }
-  __syncthreads();
-  if (tid < 32) {
-    for (int qh = 0; qh < G; ++qh) {
-      float mx = -INFINITY;
-      for (int t = tid; t < n; t += 32) mx = fmaxf(mx, sc[qh][t]);
-      for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      float s = 0.0f;
-      for (int t = tid; t < n; t += 32) s += ex2_approx(sc[qh][t] - mx);
+  float qr[DEC_GMAX][4];
+#pragma unroll
+  for (int qh = 0; qh < DEC_GMAX; ++qh)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) qr[qh][i] = qh < G ? qs[qh][4 * lane + i] : 0.0f;
+  for (int t = warp; t < n; t += 4) {
+    const uint2 u = *reinterpret_cast<const uint2 *>(kb + (int64_t)t * kD + 4 * lane);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&u.x));
+    const float2 c = __half22float2(*reinterpret_cast<const __half2 *>(&u.y));
+#pragma unroll
+    for (int qh = 0; qh < DEC_GMAX; ++qh) {
+      if (qh >= G) break;
+      float s = fmaf(qr[qh][3], c.y, fmaf(qr[qh][2], c.x, fmaf(qr[qh][1], a.y, qr[qh][0] * a.x)));
+#pragma unroll
       for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-      if (tid == 0) {
-        red[qh][0] = mx;
-        red[qh][1] = s;
+      if (lane == 0) {
+        pr[qh][t] = s * p.c2;
+        if (li == p.score_li) p.logit[((int64_t)b * p.H_q + h * G + qh) * p.block + t] = s * p.c2;
       }
     }
   }
   __syncthreads();
+  for (int qh = warp; qh < G; qh += 4) {
+    float mx = -INFINITY;
+    for (int t = lane; t < n; t += 32) mx = fmaxf(mx, pr[qh][t]);
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    float sum = 0.0f;
+    for (int t = lane; t < n; t += 32) {
+      const float e = ex2_approx(pr[qh][t] - mx);
+      pr[qh][t] = e;
+      sum += e;
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if (lane == 0) {
+      red[qh][0] = mx;
+      red[qh][1] = sum;
+    }
+  }
+  __syncthreads();
+  float o[DEC_GMAX];
+#pragma unroll
+  for (int qh = 0; qh < DEC_GMAX; ++qh) o[qh] = 0.0f;
+#pragma unroll 4
+  for (int t = 0; t < n; ++t) {
+    const float vv = __half2float(__ushort_as_half(vb[(int64_t)t * kD + tid]));
+#pragma unroll
+    for (int qh = 0; qh < DEC_GMAX; ++qh)
+      if (qh < G) o[qh] = fmaf(pr[qh][t], vv, o[qh]);
+  }
   float *dst = p.part + ((int64_t)slab * p.NU + p.unit) * G * PART_STRIDE;
-  for (int qh = 0; qh < G; ++qh) {
-    const float mx = red[qh][0];
-    float o = 0.0f;
-    if (n > 0)
-      for (int t = 0; t < n; ++t)
-        o = fmaf(ex2_approx(sc[qh][t] - mx), __half2float(__ushort_as_half(vb[(int64_t)t * kD + tid])), o);
-    dst[qh * PART_STRIDE + 4 + tid] = o;
+#pragma unroll
+  for (int qh = 0; qh < DEC_GMAX; ++qh) {
+    if (qh >= G) break;
+    dst[qh * PART_STRIDE + 4 + tid] = o[qh];
     if (tid == 0) {
-      dst[qh * PART_STRIDE + 0] = n > 0 ? mx : -INFINITY;
+      dst[qh * PART_STRIDE + 0] = n > 0 ? red[qh][0] : -INFINITY;
       dst[qh * PART_STRIDE + 1] = n > 0 ? red[qh][1] : 0.0f;
     }
   }
@@ -687,11 +715,8 @@ static int pool_smem_bytes(int G) {
 template <int L, bool ROT>
 static cudaError_t launch_pool(const DecParams &p, int grid, cudaStream_t st) {
   const int smem = pool_smem_bytes<L>(p.G);
-  cudaError_t e = cudaFuncSetAttribute(decode_pool_kernel<L, ROT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       pool_smem_bytes<L>(DEC_GMAX));
-  if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(decode_pool_kernel<L, ROT>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                           cudaSharedmemCarveoutMaxShared);
+  cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(decode_pool_kernel<L, ROT>),
+                                 pool_smem_bytes<L>(DEC_GMAX));
   if (e != cudaSuccess) return e;
   decode_pool_kernel<L, ROT><<<grid, DEC_WARPS * 32, smem, st>>>(p);
   return cudaGetLastError();
@@ -725,9 +750,7 @@ static cudaError_t launch_pool_any(int L, const DecParams &p, int grid, cudaStre
 
 // splits per slab for a pool of capacity cap (host knows only capacities)
 static int pool_splits(const semkv_cache &c, int n_layers, int cap) {
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   const int64_t slabs = (int64_t)c.B * n_layers * c.H;
   // about 1.75 waves of the 4 resident CTAs per SM, rounded to the nearest
   // split count: on the 32-layer prefill cache (256 slabs) 4 splits took
@@ -768,6 +791,7 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int sc
   p.part = reinterpret_cast<float *>(ws);
   p.NU = NU;
   p.status = status;
+  p.wait0 = first_wait_polls(kWaitLimit);
   cudaError_t e;
   // high pool
   p.kw = c.k_high; p.vw = c.v_high;

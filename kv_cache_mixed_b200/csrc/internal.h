@@ -8,6 +8,17 @@
 
 namespace semkv {
 
+// Poll bound of the first wait of each warp's bulk-copy ring: `dflt` unless a
+// test lowered it with semkv_set_first_copy_wait_polls.
+int first_wait_polls(int dflt);
+
+// Per-device host caches (devinfo.cu): SMs of the current device; set a
+// kernel's dynamic shared-memory limit (and the max-shared carveout) once per
+// device; its resident CTAs per SM for a launch shape, queried once.
+int device_sm_count();
+cudaError_t prepare_kernel(const void *fn, int smem_bytes);
+cudaError_t kernel_occupancy(const void *fn, int threads, int smem_bytes, int *ctas_per_sm);
+
 // Slot of each token within its class, and the high count per sequence.
 //   slot int32 [B][T_max], cnt_high int32 [B].
 cudaError_t launch_slot_scan(const uint8_t *mask, int64_t mask_bstride, const int32_t *seq_len,

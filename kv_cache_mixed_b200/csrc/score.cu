@@ -76,9 +76,7 @@ key_l2_kernel(const uint16_t *__restrict__ k, int64_t kbs, const int32_t *__rest
 cudaError_t launch_score_key_l2(const uint16_t *k, int64_t k_bstride, const int32_t *seq_len,
                                 int B, int T_max, int H, float *score, uint32_t *status,
                                 cudaStream_t st) {
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   const int64_t ntok = (int64_t)B * T_max;
   int64_t want = (ntok + KL2_WARPS - 1) / KL2_WARPS;
   int64_t cap = (int64_t)sms * 8;
@@ -513,6 +511,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   const int ncol_half = Np / 2;                    // pass 2: rows per warp half (Np is a multiple of 64)
   bool lost = false;
   int nwait = 0;                                   // completed phases, per accumulator
+  int pend = 0;                                    // accumulators with a commit not yet waited for
 
   for (int tile = tb; tile <= te; ++tile) {
     // issue tile `tile` (if any): its keys were staged two iterations ago
@@ -525,13 +524,18 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
         tc_fence_after();
         issue_mma(tile);
       }
+      pend |= 1 << (tile & 1);
     }
     // epilogue of tile-1
     const int et = tile - 1;
     if (et >= tb) {
       const int ab = et & 1;
-      if (mbar_wait(&bars[ab], (nwait >> ab) & 1, kUmmaWait)) nwait ^= 1 << ab;
-      else lost = true;
+      if (mbar_wait(&bars[ab], (nwait >> ab) & 1, kUmmaWait)) {
+        nwait ^= 1 << ab;
+        pend &= ~(1 << ab);
+      } else {
+        lost = true;
+      }
       tc_fence_after();
       const int t0 = et * UA_KEYS;
       const bool edge = t0 + UA_KEYS - 1 > len - p.w;
@@ -609,9 +613,12 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   }
   cp_async_wait<0>();
   if (__syncthreads_or(lost) && tid == 0) {
-    // drain: wait (bounded) for whatever MMAs are still in flight before TMEM is freed
+    // drain: wait, with the full bound, for the commit of every accumulator
+    // that still has MMAs in flight (the one whose wait gave up and the tile
+    // issued just before) before TMEM is freed
     set_flag(p.status, SEMKV_FLAG_TIMEOUT);
-    for (int ab = 0; ab < 2; ++ab) mbar_wait(&bars[ab], (nwait >> ab) & 1, kUmmaWait / 64);
+    for (int ab = 0; ab < 2; ++ab)
+      if (pend & (1 << ab)) mbar_wait(&bars[ab], (nwait >> ab) & 1, kUmmaWait);
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -660,9 +667,7 @@ cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const u
   p.Rg = p.G * w;
   p.nrb = (p.Rg + AM_ROWS - 1) / AM_ROWS;
   const int ntile = (T_max + AM_TILE - 1) / AM_TILE;
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int sms = device_sm_count();
   p.c1 = kLog2e / sqrtf((float)kD);
   const int64_t rows = (int64_t)B * H_q * w;
   const int nchunk_ws = ntile < 64 ? ntile : 64;
@@ -680,9 +685,9 @@ cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const u
     int nch = sms / (H * B);                  // whole waves only
     nch = nch < 1 ? 1 : (nch > utiles ? utiles : (nch > 64 ? 64 : nch));
     p.nchunk = nch;
-    e = cudaFuncSetAttribute(attn_umma_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, UA_SMEM);
+    e = prepare_kernel(reinterpret_cast<const void *>(attn_umma_kernel<1>), UA_SMEM);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(attn_umma_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, UA_SMEM);
+    e = prepare_kernel(reinterpret_cast<const void *>(attn_umma_kernel<2>), UA_SMEM);
     if (e != cudaSuccess) return e;
     attn_umma_kernel<1><<<dim3(nch, H, B), UA_THREADS, UA_SMEM, st>>>(p, Np, nch, head_part);
     e = cudaGetLastError();

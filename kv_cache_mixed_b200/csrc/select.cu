@@ -177,19 +177,13 @@ select_kernel(const float *__restrict__ score, int64_t score_bstride,
   }
 }
 
-static int g_sel_smem_set = 0;
-
 cudaError_t launch_select(const float *score, int64_t score_bstride, const int32_t *seq_len,
                           int len_const, int B, int T_max, int r_ppm, uint8_t *mask,
                           int64_t mask_bstride, uint32_t *status, cudaStream_t st) {
   const int cache = T_max <= SEL_SMEM_KEYS ? 1 : 0;
   const size_t smem = cache ? (size_t)T_max * 4 : 0;
-  if (!g_sel_smem_set) {
-    cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         SEL_SMEM_KEYS * 4);
-    if (e != cudaSuccess) return e;
-    g_sel_smem_set = 1;
-  }
+  cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(select_kernel), SEL_SMEM_KEYS * 4);   // once per device
+  if (e != cudaSuccess) return e;
   select_kernel<<<B, SEL_THREADS, smem, st>>>(score, score_bstride, seq_len, len_const, T_max,
                                               r_ppm, mask, mask_bstride, status, cache);
   return cudaGetLastError();
