@@ -604,7 +604,7 @@ def run_long(args, rank, world, dist):
     nh_max = kv.semkv_num_high(T, max(synth.R_SWEEP_PPM))
     nl_max = T - kv.semkv_num_high(T, min(synth.R_SWEEP_PPM))
     cache = kv.MixedCache(B, Lyr, H, H_q, wl.L_high, wl.L_low, wl.r_ppm, nh_max + 16, nl_max + 16)
-    qs = [synth.decode_query(wl, 0, s, dev) for s in range(64)]
+    qs = [synth.decode_query(wl, 0, dev, step=s) for s in range(64)]
     out = torch.empty_like(qs[0])
     fp16_in = 2 * B * Lyr * H * T * 256
     per_r = {}
@@ -666,7 +666,7 @@ def run_levels(args, rank, world, dist):
     mask = torch.empty((B, T), dtype=torch.uint8, device=dev)
     kv.semkv_score(kv.SCORE_ATTN_MASS, k[:, 0], k.stride(0), q_win, seq_len, B, T, H, H_q, w, score)
     kv.semkv_select(score, seq_len, wl.r_ppm, mask)
-    q = synth.decode_query(wl, 0, 0, dev)
+    q = synth.decode_query(wl, 0, dev)
     out = torch.empty_like(q)
     fp16_in = 2 * B * Lyr * H * T * 256
     nh = kv.semkv_num_high(T, wl.r_ppm)
@@ -852,7 +852,11 @@ def run_case(args):
     kv.semkv_select(score, seq_len, wl.r_ppm, mask)
     kv.semkv_quantize(cache, k, v, seq_len, mask)
     torch.cuda.synchronize()
-    for _ in range(args.warmup + args.steps):
+    stream = torch.cuda.current_stream()
+    times = []
+    for i in range(args.warmup + args.steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
         if args.case == "score":
             kv.semkv_score(kv.SCORE_ATTN_MASS, k[:, Lyr - 1], k.stride(0), q_win, seq_len, B, T, H, H_q, w, score)
         elif args.case == "select":
@@ -863,9 +867,13 @@ def run_case(args):
             kv.semkv_quantize(cache, k, v, seq_len, mask)
         else:
             kv.semkv_decode_attn(cache, 0, Lyr, qdec, out)
-    torch.cuda.synchronize()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            times.append(a.elapsed_time(b))
     assert cache.status_flags() == 0
-    print(json.dumps({"case": args.case, "layers": Lyr, "ok": True}))
+    print(json.dumps({"case": args.case, "layers": Lyr, "ok": True,
+                      "ms_median": round(statistics.median(times), 4) if times else None}))
 
 
 def main():

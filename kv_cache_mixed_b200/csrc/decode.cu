@@ -6,18 +6,23 @@
 //   q . khat_j = scale_j * (q . c_j) + mn_j * sum(q)
 //   sum_j p_j vhat_j = sum_j (p_j scale_j) c_j + (sum_j p_j mn_j) * 1
 // Both dot products run on tensor cores (mma.sync m16n8k16, f16 x f16 -> f32).
-// Codes enter the tensor cores as raw f16 subnormal bit patterns c * 2^-24
-// (exact), so a digit costs no conversion: unpacking a 32-bit word gives the
-// digit in the low bits of a register and two digits packed in one register
-// are already an f16x2 operand.  The 2^24 factor is folded into the scales.
+// Two digits of one token sit in one f16x2 register, which is the operand
+// format of the MMA, so a digit is never converted after it is extracted.
 //
-// Digit extraction (any L in [2,16]): a word is split by constant divisors into
-// parts of k digits with L^k small enough that, with F = v * ceil(2^32/L^k),
-// each step t = F * L yields the next digit (most significant first) in the
-// high 32 bits and the next F in the low 32 bits.  The part sizes below were
-// checked exhaustively against repeated division for every part value.  For
-// L <= 6 one step by L^2 yields two digits, turned into the f16x2 operand by a
-// small shared-memory table.
+// Digit extraction, levels that are not powers of two: a word is cut by
+// integer division into parts of k digits (L^k <= 1024), and two parts are
+// packed into one f16x2 register as the exact values 1024 + P (bit pattern
+// 0x6400 + P).  Then, on both halves at once, one f16 step
+//     t = fma(X, c, K)                 = 1536 + floor(P / L)   (exact; c, K below)
+//     digit = X + fma(t, -L, 1536 L - B) = P - L floor(P / L)   (exact)
+// peels the least significant digit off, and t is the next step's X (B is
+// X's bias: 1024 first, then 1536).  Every value stays an integer below 2048,
+// so each f16 operation is exact; (c, K) were chosen so that the rounding of
+// X c + K lands on 1536 + floor(P / L) for every part value, checked
+// exhaustively.  A step is three f16x2 instructions for two digits, all on
+// the FMA pipe.  Levels that are powers of two (2, 4, 8, 16) take their
+// digits straight out of the bit fields instead, as f16 subnormal patterns
+// c * 2^-24 (exact), with the 2^24 folded into the scales.
 //
 // Work split: one pool class per launch (template on its L, and on whether
 // the rows are Hadamard-rotated); CTA = 4 warps on a contiguous range of
@@ -31,182 +36,224 @@
 // MMA shapes per 16-token tile: the logits put the 16 tokens on the MMA rows
 // and the query heads on the 8 columns (one m16n8k16 per 16 head-dim slots);
 // the values put 16 head-dim slots on the rows and the query heads on the
-// columns, with P' moved into that operand layout by movmatrix.  With at most
-// 4 query heads per KV head, columns 4..7 of the value MMA carry the low f16
-// part of P', so one MMA takes both parts.
+// columns, with the digits and P' moved into that operand layout by
+// movmatrix.  With at most 4 query heads per KV head, columns 4..7 of the
+// value MMA carry the low f16 part of P', so one MMA takes both parts.
 #include "common.cuh"
 #include "internal.h"
 
 namespace semkv {
 
 constexpr int DEC_WARPS = 4;
-constexpr int DEC_NST = 4;                  // tiles in flight per warp
+constexpr int DEC_NST = 3;                  // 32-token tiles in flight per warp
 constexpr int DEC_GMAX = 8;                 // query heads per KV head handled (M rows used)
 constexpr int PART_STRIDE = 132;            // floats per partial: m, l, pad, pad, o[128]
 constexpr float kLog2eF = 1.4426950408889634f;
 
-// ---- digit split table: part sizes in digits, least significant part first
-__host__ __device__ constexpr int split_part(int L, int i) {
-  // {part0, part1, part2} per L; a 0 marks an unused part
-  return L == 2 ? (i < 2 ? 16 : 0) : L == 3 ? (i < 2 ? 10 : 0) : L == 4 ? (i < 2 ? 8 : 0)
-       : L == 5 ? (i == 0 ? 6 : i == 1 ? 7 : 0) : L == 6 ? (i < 2 ? 6 : 0)
-       : L == 7 ? (i == 0 ? 3 : 4) : L == 8 ? (i < 2 ? 5 : 0) : L == 9 ? (i < 2 ? 5 : 0)
-       : L == 10 ? (i == 0 ? 4 : i == 1 ? 5 : 0) : L == 11 ? 3 : (i < 2 ? 4 : 0);
-}
-__host__ __device__ constexpr int split_parts(int L) { return (L == 7 || L == 11) ? 3 : 2; }
+__host__ __device__ constexpr bool is_pow2_level(int L) { return L == 2 || L == 4 || L == 8 || L == 16; }
 
-// Pair path (L <= 6): one wide multiply by L^2 yields two digits at once,
-// hi = c_{j+1} * L + c_j, and a shared-memory table of L^2 entries turns hi
-// into the f16x2 operand (c_j, c_{j+1}).  Every part of these levels starts on
-// an even digit and only the top part can have odd length, so with the word
-// stride in slots rounded up to even (L = 5: 13 digits in 14 slots) every pair
-// stays inside one part; an odd top part leads with one single-digit step.
-__host__ __device__ constexpr bool use_pairs(int L) { return L <= 6; }
+// ---- f16 digit plan of a level that is not a power of two: part sizes in
+// digits (least significant part first; consecutive parts share a register)
+// and the f16 bit patterns of (c, K) for the first step (X = 1024 + P) and
+// for the later steps (X = 1536 + P).
+struct F16Plan {
+  int np;
+  int part[5];
+  uint16_t c0, k0, c1, k1;
+};
+__host__ __device__ constexpr F16Plan f16_plan(int L) {
+  return L == 3    ? F16Plan{4, {5, 5, 5, 5, 0}, 0x3553, 0x64ab, 0x3552, 0x6401}
+         : L == 5  ? F16Plan{4, {4, 4, 3, 2, 0}, 0x3265, 0x6533, 0x3263, 0x64cd}
+         : L == 6  ? F16Plan{4, {3, 3, 3, 3, 0}, 0x3155, 0x6555, 0x3153, 0x6500}
+         : L == 7  ? F16Plan{4, {3, 3, 3, 2, 0}, 0x3094, 0x656d, 0x3093, 0x6524}
+         : L == 9  ? F16Plan{5, {2, 2, 2, 2, 2}, 0x2f19, 0x658e, 0x2ee6, 0x655a}
+         : L == 10 ? F16Plan{4, {3, 2, 2, 2, 0}, 0x2e68, 0x6599, 0x2e66, 0x6566}
+         : L == 11 ? F16Plan{5, {2, 2, 2, 2, 1}, 0x2dc9, 0x65a3, 0x2da6, 0x6578}
+         : L == 12 ? F16Plan{4, {2, 2, 2, 2, 0}, 0x2d58, 0x65aa, 0x2d26, 0x6584}
+         : L == 13 ? F16Plan{4, {2, 2, 2, 2, 0}, 0x2ce9, 0x65b1, 0x2cc6, 0x658d}
+         : L == 14 ? F16Plan{4, {2, 2, 2, 2, 0}, 0x2c98, 0x65b6, 0x2c66, 0x6596}
+         : L == 15 ? F16Plan{4, {2, 2, 2, 2, 0}, 0x2c48, 0x65bb, 0x2c3b, 0x659a}
+                   : F16Plan{0, {0, 0, 0, 0, 0}, 0, 0, 0, 0};
+}
+__host__ __device__ constexpr int plan_part(int L, int i) { return i < f16_plan(L).np ? f16_plan(L).part[i] : 0; }
+__host__ __device__ constexpr int plan_regs(int L) { return (f16_plan(L).np + 1) / 2; }
+__host__ __device__ constexpr int plan_steps(int L, int j) {
+  return f16_plan(L).part[2 * j] > (2 * j + 1 < f16_plan(L).np ? f16_plan(L).part[2 * j + 1] : 0)
+             ? f16_plan(L).part[2 * j]
+             : f16_plan(L).part[2 * j + 1];
+}
+__host__ __device__ constexpr int plan_offset(int L, int i) {
+  int o = 0;
+  for (int m = 0; m < i; ++m) o += f16_plan(L).part[m];
+  return o;
+}
+
+// f16x2 registers (digit pairs) one word yields
+__host__ __device__ constexpr int word_regs(int L) {
+  if (is_pow2_level(L)) return digits_per_word(L) / 2;
+  int r = 0;
+  for (int j = 0; j < plan_regs(L); ++j) r += plan_steps(L, j);
+  return r;
+}
+// digit (within the word) in half `h` (0 = low, 1 = high) of register m, or -1 (padding)
+__host__ __device__ constexpr int reg_digit(int L, int m, int h) {
+  if (is_pow2_level(L)) return m + h * (digits_per_word(L) / 2);
+  int base = 0;
+  for (int j = 0; j < plan_regs(L); ++j) {
+    const int st = plan_steps(L, j);
+    if (m < base + st) {
+      const int pi = 2 * j + h, s = m - base;
+      if (pi >= f16_plan(L).np || s >= f16_plan(L).part[pi]) return -1;
+      return plan_offset(L, pi) + s;
+    }
+    base += st;
+  }
+  return -1;
+}
 
 template <int L>
 struct Geo {
   static constexpr int N = digits_per_word(L);       // digits per word
   static constexpr int W = words_per_row(L);         // words per row
-  static constexpr int S = use_pairs(L) ? N + (N & 1) : N;   // slots per word
+  static constexpr int S = 2 * word_regs(L);         // digit slots per word
+  static constexpr int SP = (S + 3) / 4 * 4;         // slots per word, padded to whole k-block positions
+  static constexpr int RPW = SP / 2;                 // f16x2 registers per word
+  static constexpr int KPW = SP / 4;                 // k-blocks per word
   static constexpr int WPG = (W + 3) / 4;            // words per lane group (lane % 4)
-  static constexpr int KB = (WPG * S + 3) / 4;       // 16-slot k-blocks
-  static constexpr int TILE_BYTES = 16 * W * 4 * 2 + 16 * 8 * 2;
-  static_assert(split_part(L, 0) + split_part(L, 1) + split_part(L, 2) == N, "split must cover the word");
-  static_assert(!use_pairs(L) || (split_part(L, 0) % 2 == 0 && (split_parts(L) == 2 || split_part(L, 1) % 2 == 0)),
-                "pair path needs even parts below the top part");
+  static constexpr int KB = WPG * KPW;               // 16-slot k-blocks
+  static constexpr int TT = 32;                      // tokens per tile (two 16-token MMA blocks)
+  static constexpr int TILE_BYTES = TT * W * 4 * 2 + TT * 8 * 2;
+  // digits are f16 subnormal patterns c * 2^-24 on the bit-field path
+  static constexpr float FAC = is_pow2_level(L) ? 16777216.0f : 1.0f;
 };
 
-// digit j (0 = least significant) of word w into dig[j0 + j].  Lr holds L at
-// run time so that every digit step stays one wide multiply.
-template <int L, int NDIG>
-__device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&dig)[NDIG], int j0, uint32_t Lr) {
-  constexpr int NP = split_parts(L);
-  uint32_t rest = w;
-  int jb = j0;
-#pragma unroll
-  for (int pi = 0; pi < NP; ++pi) {
-    const int k = split_part(L, pi);
-    uint32_t v;
-    if (pi < NP - 1) {
-      const uint32_t P = (uint32_t)ipow(L, k);
-      const uint32_t qq = rest / P;
-      v = rest - qq * P;
-      rest = qq;
-    } else {
-      v = rest;
-    }
-    const uint32_t M = (uint32_t)(((1ull << 32) + ipow(L, k) - 1) / ipow(L, k));
-    uint32_t F = v * M;
-#pragma unroll
-    for (int d = k - 1; d >= 0; --d) {
-      uint32_t lo, hi;
-      mul_wide(F, Lr, lo, hi);
-      dig[jb + d] = hi;
-      F = lo;
-    }
-    jb += k;
-  }
+__device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+__device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__host__ __device__ constexpr uint32_t h2dup(uint16_t b) { return (uint32_t)b | ((uint32_t)b << 16); }
+// f16 bits of a small integer v (|v| < 2^15, exactly representable)
+__host__ __device__ constexpr uint16_t f16_int_bits(int v) {
+  int a = v < 0 ? -v : v;
+  int e = 0;
+  while ((a >> (e + 1)) != 0) ++e;                   // a in [2^e, 2^(e+1))
+  const int mant = e >= 10 ? (a >> (e - 10)) & 0x3ff : (a << (10 - e)) & 0x3ff;
+  return (uint16_t)((v < 0 ? 0x8000 : 0) | ((e + 15) << 10) | mant);
 }
 
-// pair path: f16x2 registers of slot pairs (j0 + 2m, j0 + 2m + 1) into pr[j0/2 + m]
-template <int L, int NPR>
-__device__ __forceinline__ void extract_word_pairs(uint32_t w, uint32_t (&pr)[NPR], int j0, uint32_t Lr,
-                                                   uint32_t L2r, const uint32_t *lut) {
-  constexpr int NP = split_parts(L);
-  uint32_t rest = w;
-  int jb = j0;
+// the S/2 digit-pair registers of word w, in slot order, into out[o0 ..]
+template <int L, int NR>
+__device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&out)[NR], int o0) {
+  if constexpr (L == 2 || L == 4 || L == 16) {
+    constexpr int b = L == 2 ? 1 : (L == 4 ? 2 : 4);
+    constexpr uint32_t msk = (uint32_t)(L - 1) * 0x00010001u;
 #pragma unroll
-  for (int pi = 0; pi < NP; ++pi) {
-    const int k = split_part(L, pi);
-    uint32_t v;
-    if (pi < NP - 1) {
-      const uint32_t P = (uint32_t)ipow(L, k);
-      const uint32_t qq = rest / P;
-      v = rest - qq * P;
-      rest = qq;
-    } else {
-      v = rest;
-    }
-    const uint32_t M = (uint32_t)(((1ull << 32) + ipow(L, k) - 1) / ipow(L, k));
-    uint32_t F = v * M;
-    if (k & 1) {                       // odd top part: its top digit alone, upper half zero
-      uint32_t lo, hi;
-      mul_wide(F, Lr, lo, hi);
-      pr[(jb + k - 1) >> 1] = hi;
-      F = lo;
-    }
+    for (int m = 0; m < 16 / b; ++m) out[o0 + m] = (w >> (b * m)) & msk;   // digits m, m + 16/b
+  } else if constexpr (L == 8) {
+    out[o0] = (w & 7u) | ((w << 1) & 0x70000u);                              // digits 0, 5
 #pragma unroll
-    for (int m = k / 2 - 1; m >= 0; --m) {
-      uint32_t lo, hi;
-      mul_wide(F, L2r, lo, hi);
-      pr[(jb >> 1) + m] = lut[hi];
-      F = lo;
+    for (int m = 1; m < 5; ++m) out[o0 + m] = ((w >> (3 * m)) & 7u) | ((w >> (3 * m - 1)) & 0x70000u);
+  } else {
+    constexpr uint32_t C0 = h2dup(f16_plan(L).c0), K0 = h2dup(f16_plan(L).k0);
+    constexpr uint32_t C1 = h2dup(f16_plan(L).c1), K1 = h2dup(f16_plan(L).k1);
+    constexpr uint32_t NEGL = h2dup(f16_int_bits(-L));
+    constexpr uint32_t R0 = h2dup(f16_int_bits(1536 * L - 1024)), R1 = h2dup(f16_int_bits(1536 * L - 1536));
+    constexpr uint32_t M1024 = h2dup(f16_int_bits(-1024)), M1536 = h2dup(f16_int_bits(-1536));
+    uint32_t rest = w;
+    int o = o0;
+#pragma unroll
+    for (int j = 0; j < plan_regs(L); ++j) {
+      const int ka = plan_part(L, 2 * j);
+      const int kb = plan_part(L, 2 * j + 1);
+      uint32_t v;
+      if (j < plan_regs(L) - 1) {
+        const uint32_t D = (uint32_t)ipow(L, ka + kb);
+        const uint32_t qq = rest / D;
+        v = rest - qq * D;
+        rest = qq;
+      } else {
+        v = rest;
+      }
+      uint32_t x;
+      if (kb > 0) {
+        // (v mod L^ka) | (v div L^ka) << 16: the quotient by multiply-high is
+        // exact because v < L^(ka+kb) and L^ka * L^(ka+kb) < 2^32
+        const uint32_t Da = (uint32_t)ipow(L, ka);
+        const uint32_t q = __umulhi(v, (uint32_t)((0x100000000ull + Da - 1) / Da));
+        x = (v + q * (65536u - Da)) | 0x64006400u;
+      } else {
+        x = v | 0x64006400u;
+      }
+      const int st = ka > kb ? ka : kb;
+      if (st == 1) {
+        out[o++] = hadd2(x, M1024);
+        continue;
+      }
+      uint32_t t = hfma2(x, C0, K0);
+      out[o++] = hadd2(x, hfma2(t, NEGL, R0));
+#pragma unroll
+      for (int s = 1; s < st - 1; ++s) {
+        const uint32_t t2 = hfma2(t, C1, K1);
+        out[o++] = hadd2(t, hfma2(t2, NEGL, R1));
+        t = t2;
+      }
+      out[o++] = hadd2(t, M1536);
     }
-    jb += k;
   }
 }
 
 // The lane group c = lane % 4 owns words c*WPG .. c*WPG+WPG-1 of a token row.
-// Its digit slot u = i*S + j (word i, digit j) sits in k-block u/4 at
-// position u%4; positions 0,1 are one f16x2 register, 2,3 the other.
+// Its digit slot u = i*SP + j (word i, slot j) sits in k-block u/4 at position
+// u%4; positions 0,1 are one f16x2 register, 2,3 the other.  Word i alone
+// fills k-blocks i*KPW .. i*KPW+KPW-1, so a word's registers can go to the
+// tensor cores as soon as it is unpacked.  Words past W of the row read the
+// next bytes of the tile buffer: every part of any 32-bit value stays a
+// finite f16, and those slots carry q = 0 (K) or are never written out (V).
 template <int L>
-__device__ __forceinline__ void unpack_row(const uint32_t *wrow, int c, uint32_t Lr, uint32_t L2r,
-                                           const uint32_t *lut, uint32_t (&reg)[Geo<L>::KB][2]) {
-  using G = Geo<L>;
-  constexpr int ND = G::KB * 4;
-  // words past W of the row read the next bytes of the tile buffer: any 32-bit
-  // value unpacks to digits in [0, L) and those slots carry q = 0 (K) or are
-  // never written out (V), so no bounds check is needed
-  const uint32_t *wr = wrow + c * G::WPG;
-  if constexpr (use_pairs(L)) {
-    uint32_t pr[ND / 2];
+__device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&reg)[Geo<L>::RPW]) {
+  extract_word<L, Geo<L>::RPW>(w, reg, 0);
 #pragma unroll
-    for (int i = 0; i < G::WPG; ++i) extract_word_pairs<L, ND / 2>(wr[i], pr, i * G::S, Lr, L2r, lut);
-#pragma unroll
-    for (int u = (G::WPG * G::S) / 2; u < ND / 2; ++u) pr[u] = 0u;
-#pragma unroll
-    for (int kb = 0; kb < G::KB; ++kb) {
-      reg[kb][0] = pr[2 * kb];
-      reg[kb][1] = pr[2 * kb + 1];
-    }
-  } else {
-    uint32_t dig[ND];
-#pragma unroll
-    for (int i = 0; i < G::WPG; ++i) extract_word<L, ND>(wr[i], dig, i * G::N, Lr);
-#pragma unroll
-    for (int u = G::WPG * G::N; u < ND; ++u) dig[u] = 0u;
-#pragma unroll
-    for (int kb = 0; kb < G::KB; ++kb) {
-      reg[kb][0] = __byte_perm(dig[4 * kb], dig[4 * kb + 1], 0x5410);
-      reg[kb][1] = __byte_perm(dig[4 * kb + 2], dig[4 * kb + 3], 0x5410);
-    }
-  }
+  for (int u = Geo<L>::S / 2; u < Geo<L>::RPW; ++u) reg[u] = 0u;
 }
 
 // head-dim index of slot u of lane group c (or -1 for a padding slot)
 template <int L>
 __device__ __forceinline__ int slot_dim(int c, int u) {
   using G = Geo<L>;
-  const int wi = c * G::WPG + u / G::S;
-  const int j = u % G::S;
-  const int d = wi * G::N + j;
-  return (u < G::WPG * G::S && j < G::N && wi < G::W && d < kD) ? d : -1;
+  const int wi = c * G::WPG + u / G::SP;
+  const int j = u % G::SP;
+  const int dg = j < G::S ? reg_digit(L, j >> 1, j & 1) : -1;
+  const int d = wi * G::N + dg;
+  return (u < G::WPG * G::SP && dg >= 0 && wi < G::W && d < kD) ? d : -1;
 }
 
-struct DecParams {
-  // pool of this launch
+// one pool class of a launch
+struct PoolArgs {
   const uint32_t *kw, *vw;          // [B][Lyr][H][cap][W]
   const float2 *km, *vm;            // [B][Lyr][H][cap]
   const int32_t *count;             // [B]
   int cap;
+  int S, unit0;                     // splits per slab, first partial unit of this class
+};
+
+struct DecParams {
+  // the classes of this launch: CTAs [0, slabs*pool[0].S) take class 0, the
+  // next slabs*pool[1].S take class 1 (pool[1].S = 0 when a launch has one class)
+  PoolArgs pool[2];
+  int slabs;
   // cache geometry
   int B, Lyr, H, H_q, G, layer0, nL;
   const uint16_t *q;                // [B][nL][H_q][D]
   float c2;                         // sm_scale * log2(e)
   float *part;                      // [slabs][NU][G][PART_STRIDE]
-  int NU, unit0, S;                 // units per slab, first unit of this launch, splits
+  int NU;                           // partial units per slab
   uint32_t *status;
-  uint32_t Lrt;                     // the pool's level count (equals the template L)
   int rot;                          // rows stored Hadamard-rotated (needs G <= 4)
   int wait0;                        // polls of each warp's first copy wait (testing aid)
 };
@@ -220,38 +267,31 @@ constexpr int kQOff = kBarOff<L> + DEC_WARPS * DEC_NST * 8;
 static_assert(Geo<6>::TILE_BYTES % 16 == 0 && Geo<5>::TILE_BYTES % 16 == 0 && kMergeBytes % 16 == 0,
               "tile buffers must keep 16-byte alignment for bulk copies");
 constexpr int kWaitLimit = 1 << 20;         // mbarrier polls before a copy is declared lost
-constexpr int kLutBytes = 64 * 4;           // pair table, L*L <= 36 entries
 template <int L>
 constexpr int kQfragBytes = Geo<L>::KB * 32 * 8;   // q operand fragments, [kb][lane] x 2 words
 
+// One CTA's share of one pool class: tiles [tb, te) of split `split` of slab `slab`.
 template <int L, bool ROT>
-__global__ void __launch_bounds__(DEC_WARPS * 32, 4)
-decode_pool_kernel(const DecParams p) {
+__device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa, int slab, int split,
+                                          uint8_t *smem) {
   using Gm = Geo<L>;
   constexpr int KB = Gm::KB, W = Gm::W;
   constexpr float kappa = (L == 2) ? 0.5f : 1.0f;       // keeps p*scale inside f16 range
-  extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
-  const int slab = blockIdx.x / p.S, split = blockIdx.x % p.S;
   const int h = slab % p.H, li = (slab / p.H) % p.nL, b = slab / (p.H * p.nL);
   const int64_t pslab = ((int64_t)b * p.Lyr + p.layer0 + li) * p.H + h;
   const int G = p.G;
-  const uint32_t Lr = p.Lrt;                             // == L, opaque to the compiler
-  const uint32_t L2r = Lr * Lr;
 
   // ---- shared memory: per-warp tile rings, their mbarriers, then the q rows
   uint8_t *ring = smem + warp * DEC_NST * Gm::TILE_BYTES;
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff<L>) + warp * DEC_NST;
-  uint32_t *lut = reinterpret_cast<uint32_t *>(smem + kQOff<L>);      // [L*L] digit pairs (pair path)
-  uint2 *qfrag = reinterpret_cast<uint2 *>(smem + kQOff<L> + kLutBytes);            // [KB][32]
-  float *qs = reinterpret_cast<float *>(smem + kQOff<L> + kLutBytes + kQfragBytes<L>);  // [G][128]
+  uint2 *qfrag = reinterpret_cast<uint2 *>(smem + kQOff<L>);                        // [KB][32]
+  float *qs = reinterpret_cast<float *>(smem + kQOff<L> + kQfragBytes<L>);            // [G][128]
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < DEC_NST; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
   }
-  if (use_pairs(L))
-    for (int i = threadIdx.x; i < L * L; i += DEC_WARPS * 32) lut[i] = (uint32_t)(i % L) | ((uint32_t)(i / L) << 16);
   for (int i = threadIdx.x; i < G * kD; i += DEC_WARPS * 32) {
     const int qh = i / kD, d = i % kD;
     const uint16_t hb = p.q[(((int64_t)b * p.nL + li) * p.H_q + h * G + qh) * kD + d];
@@ -277,9 +317,11 @@ decode_pool_kernel(const DecParams p) {
   // With rotated rows q' is not an f16 value: columns 0..3 carry its f16
   // high part and columns 4..7 (G <= 4) its low part, q' - hi, so one MMA
   // gives the logit to about 2^-22 relative.
+  // Without rotation and with G <= 4, columns 4..7 repeat the query heads of
+  // columns 0..3, so every lane of a row gets the logits of its head pair.
   float qsum = 0.0f;
   const bool qlo = ROT && r >= 4;
-  const int rq = ROT ? (r & 3) : r;
+  const int rq = (ROT || G <= 4) ? (r & 3) : r;
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) {
     uint32_t qv[2];
@@ -302,38 +344,43 @@ decode_pool_kernel(const DecParams p) {
   qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
   const float c2k = ROT ? p.c2 * (1.0f / 128.0f) : p.c2;     // rotated: q' . k' / 128
   const float qsc = qsum * c2k;
-  const float kscale = c2k * 16777216.0f;              // 2^24: codes are c * 2^-24
+  const float kscale = c2k * Gm::FAC;                  // bit-field digits are c * 2^-24
   // This lane's two queries are the MMA columns 2c, 2c+1 of the logits.  With
-  // G <= 4 the value MMA's columns 4..7 carry the low f16 part of P' for
-  // queries 0..3, so lanes c >= 2 mirror the softmax of lane c-2 and one MMA
-  // per k-block takes both parts.
+  // G <= 4 columns 4..7 repeat heads 0..3 (or carry q''s low part when
+  // rotated), so lane c >= 2 holds the same two heads as lane c-2 and the two
+  // lanes split each tile's blocks; the value MMA's columns 4..7 carry the low
+  // f16 part of P', so one MMA per k-block takes both parts.
   const bool pack_lo = G <= 4;
   const int qc0 = pack_lo ? ((2 * c) & 3) : 2 * c;
   const float qs0 = __shfl_sync(0xffffffffu, qsc, 4 * qc0);        // sum(q)*c2 lives in quad r
   const float qs1 = __shfl_sync(0xffffffffu, qsc, 4 * (qc0 + 1));
 
-  // ---- this CTA's tiles
-  const int n = min(p.count[b], p.cap);
-  const int ntile = (n + 15) >> 4;
-  const int tb = (int)((int64_t)ntile * split / p.S), te = (int)((int64_t)ntile * (split + 1) / p.S);
-  const uint32_t *kw = p.kw + pslab * p.cap * W;
-  const uint32_t *vw = p.vw + pslab * p.cap * W;
-  const float2 *km = p.km + pslab * p.cap;
-  const float2 *vm = p.vm + pslab * p.cap;
+  // ---- this CTA's tiles (32 tokens each)
+  constexpr int RPW = Gm::RPW, KPW = Gm::KPW, WPG = Gm::WPG, TT = Gm::TT;
+  const int n = min(pa.count[b], pa.cap);
+  const int ntile = (n + TT - 1) / TT;
+  const int tb = (int)((int64_t)ntile * split / pa.S), te = (int)((int64_t)ntile * (split + 1) / pa.S);
+  const uint32_t *kw = pa.kw + pslab * pa.cap * W;
+  const uint32_t *vw = pa.vw + pslab * pa.cap * W;
+  const float2 *km = pa.km + pslab * pa.cap;
+  const float2 *vm = pa.vm + pslab * pa.cap;
 
   // one lane streams the warp's tiles: 4 bulk copies (K words, V words, K meta,
-  // V meta) completing on the slot's mbarrier
-  constexpr uint32_t kWB = 64 * W;                    // bytes of 16 rows of words
+  // V meta) completing on the slot's mbarrier.  Capacities are multiples of
+  // 16, so the last tile of a slab may hold 16 rows: the copies stop at the
+  // capacity, and the rows of the buffer past it are masked like rows past n.
   auto issue = [&](int tile, int slotix) {
     if (lane == 0 && tile < te) {
       uint8_t *dst = ring + slotix * Gm::TILE_BYTES;
-      const int t0 = tile * 16;
+      const int t0 = tile * TT;
+      const int nt = min(TT, pa.cap - t0);
+      const uint32_t wb = (uint32_t)nt * W * 4;
       fence_proxy_async_smem();
-      mbar_expect_tx(&bars[slotix], 2 * kWB + 256);
-      bulk_g2s(dst, kw + (int64_t)t0 * W, kWB, &bars[slotix]);
-      bulk_g2s(dst + kWB, vw + (int64_t)t0 * W, kWB, &bars[slotix]);
-      bulk_g2s(dst + 2 * kWB, km + t0, 128, &bars[slotix]);
-      bulk_g2s(dst + 2 * kWB + 128, vm + t0, 128, &bars[slotix]);
+      mbar_expect_tx(&bars[slotix], 2 * wb + (uint32_t)nt * 16);
+      bulk_g2s(dst, kw + (int64_t)t0 * W, wb, &bars[slotix]);
+      bulk_g2s(dst + TT * W * 4, vw + (int64_t)t0 * W, wb, &bars[slotix]);
+      bulk_g2s(dst + TT * W * 8, km + t0, (uint32_t)nt * 8, &bars[slotix]);
+      bulk_g2s(dst + TT * W * 8 + TT * 8, vm + t0, (uint32_t)nt * 8, &bars[slotix]);
     }
   };
 
@@ -341,6 +388,11 @@ decode_pool_kernel(const DecParams p) {
   float oacc[KB][4];
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) oacc[kb][0] = oacc[kb][1] = oacc[kb][2] = oacc[kb][3] = 0.0f;
+  // With G <= 4 the two 16-token blocks of a tile split the softmax: lanes
+  // c < 2 take block 0, lanes c >= 2 block 1 (their MMA columns duplicate the
+  // same query heads); with G > 4 every lane takes both blocks.
+  const int nb = pack_lo ? 1 : 2;
+  const int myblk = pack_lo ? (c >> 1) : 0;
 
   // ring prologue
   int next = tb + warp;
@@ -363,43 +415,70 @@ decode_pool_kernel(const DecParams p) {
     parity ^= 1u << slotix;
     const uint8_t *tbuf = ring + slotix * Gm::TILE_BYTES;
     const uint32_t *sk = reinterpret_cast<const uint32_t *>(tbuf);
-    const uint32_t *sv = reinterpret_cast<const uint32_t *>(tbuf + 64 * W);
-    const float2 *skm = reinterpret_cast<const float2 *>(tbuf + 128 * W);
-    const float2 *svm = reinterpret_cast<const float2 *>(tbuf + 128 * W + 128);
-    const int t0 = tile * 16;
+    const uint32_t *sv = reinterpret_cast<const uint32_t *>(tbuf + TT * W * 4);
+    const float2 *skm = reinterpret_cast<const float2 *>(tbuf + TT * W * 8);
+    const float2 *svm = reinterpret_cast<const float2 *>(tbuf + TT * W * 8 + TT * 8);
+    const int t0 = tile * TT;
+    const bool full = t0 + TT <= n;
 
-    // ---- logits S = C Q^T: tokens r, r+8 on the MMA rows, queries on the
-    // columns; even and odd k-blocks accumulate apart (shorter MMA chain)
-    float lg[4];                          // (token r, q0), (r, q1), (r+8, q0), (r+8, q1)
-    {
-      uint32_t ka[KB][2], kb8[KB][2];
-      unpack_row<L>(sk + r * W, c, Lr, L2r, lut, ka);
-      unpack_row<L>(sk + (8 + r) * W, c, Lr, L2r, lut, kb8);
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    // ---- logits S = C Q^T per 16-token block: tokens on the MMA rows (r, r+8),
+    // query heads on the columns; each word goes to the tensor cores as soon
+    // as it is unpacked
+    float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-      for (int kb = 0; kb < KB; ++kb) {
-        const uint2 qb = qfrag[kb * 32 + lane];
-        if (kb & 1) mma_16816(sb, ka[kb][0], kb8[kb][0], ka[kb][1], kb8[kb][1], qb.x, qb.y);
-        else mma_16816(sa, ka[kb][0], kb8[kb][0], ka[kb][1], kb8[kb][1], qb.x, qb.y);
-      }
+    for (int i = 0; i < WPG; ++i) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float sv = sa[i] + sb[i];
-        const float mirror = __shfl_xor_sync(0xffffffffu, sv, 2);
-        if (ROT) sv = sv + mirror;                    // high + low part of q'
-        else if (pack_lo && c >= 2) sv = mirror;
-        const int tt = (i < 2) ? r : 8 + r;
-        const float2 mm = skm[tt];
-        const float v = __fmaf_rn(sv, mm.y * kscale, mm.x * ((i & 1) ? qs1 : qs0));
-        lg[i] = (t0 + tt < n) ? v : -INFINITY;
+      for (int blk = 0; blk < 2; ++blk) {
+        uint32_t ra[RPW], rb[RPW];
+        unpack_word<L>(sk[(blk * 16 + r) * W + c * WPG + i], ra);
+        unpack_word<L>(sk[(blk * 16 + 8 + r) * W + c * WPG + i], rb);
+#pragma unroll
+        for (int m = 0; m < KPW; ++m) {
+          const uint2 qb = qfrag[(i * KPW + m) * 32 + lane];
+          mma_16816(sacc[blk], ra[2 * m], rb[2 * m], ra[2 * m + 1], rb[2 * m + 1], qb.x, qb.y);
+        }
       }
     }
-    // ---- online softmax (log2 domain): max over the 16 tokens = over r
-    float mx0 = fmaxf(lg[0], lg[2]), mx1 = fmaxf(lg[1], lg[3]);
+    float lg[2][4];                       // per lane block j: (token r, q0), (r, q1), (r+8, q0), (r+8, q1)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      if (j >= nb) break;
+      float s4[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float a0 = sacc[0][i], a1 = sacc[1][i];
+        if (ROT) {                                    // high + low part of q'
+          a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
+          a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+        }
+        s4[i] = (pack_lo ? myblk : j) ? a1 : a0;
+      }
+      const int tt = (pack_lo ? myblk : j) * 16 + r;
+      const float2 m0 = skm[tt], m1 = skm[tt + 8];
+      lg[j][0] = __fmaf_rn(s4[0], m0.y * kscale, m0.x * qs0);
+      lg[j][1] = __fmaf_rn(s4[1], m0.y * kscale, m0.x * qs1);
+      lg[j][2] = __fmaf_rn(s4[2], m1.y * kscale, m1.x * qs0);
+      lg[j][3] = __fmaf_rn(s4[3], m1.y * kscale, m1.x * qs1);
+      if (!full) {
+        if (t0 + tt >= n) lg[j][0] = lg[j][1] = -INFINITY;
+        if (t0 + tt + 8 >= n) lg[j][2] = lg[j][3] = -INFINITY;
+      }
+    }
+    // ---- online softmax (log2 domain): max over the tile's tokens, shared
+    // by the two lanes (c, c^2) of a head pair when they split the blocks
+    float mx0 = fmaxf(lg[0][0], lg[0][2]), mx1 = fmaxf(lg[0][1], lg[0][3]);
+    if (!pack_lo) {
+      mx0 = fmaxf(mx0, fmaxf(lg[1][0], lg[1][2]));
+      mx1 = fmaxf(mx1, fmaxf(lg[1][1], lg[1][3]));
+    }
 #pragma unroll
     for (int o = 4; o <= 16; o <<= 1) {
       mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
       mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+    }
+    if (pack_lo) {
+      mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+      mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
     }
     const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
     if (__any_sync(0xffffffffu, (mn0 > m_run[0]) | (mn1 > m_run[1]))) {
@@ -421,54 +500,72 @@ decode_pool_kernel(const DecParams p) {
     }
     // P' = p * scale * kappa as an f16 pair hi + lo (hi = RN(P'), lo = RN(P' - hi)):
     // relative error 2^-22 instead of 2^-11 for a single f16
-    uint32_t xh[2], xl[2];                // (token r | r+8): f16x2 of columns 2c, 2c+1
+    uint32_t xh[2][2], xl[2][2];          // [lane block][token r | r+8]: f16x2 of this lane's two heads
 #pragma unroll
-    for (int g2 = 0; g2 < 2; ++g2) {
-      const int tt = g2 ? 8 + r : r;
-      const bool ok = t0 + tt < n;
-      const float2 vmm = svm[tt];
-      float pw[2];
+    for (int j = 0; j < 2; ++j) {
+      if (j >= nb) break;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float pr = ok ? ex2_approx(lg[2 * g2 + e] - m_run[e]) : 0.0f;
-        l_run[e] += pr;
-        mt_run[e] += pr * vmm.x;
-        pw[e] = pr * (vmm.y * kappa);
+      for (int g2 = 0; g2 < 2; ++g2) {
+        const int tt = (pack_lo ? myblk : j) * 16 + 8 * g2 + r;
+        const bool ok = full || t0 + tt < n;
+        // rows past the count hold whatever the pool memory held: keep them out
+        const float2 vmm = ok ? svm[tt] : make_float2(0.0f, 0.0f);
+        float pw[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float pr = ok ? ex2_approx(lg[j][2 * g2 + e] - m_run[e]) : 0.0f;
+          l_run[e] += pr;
+          mt_run[e] += pr * vmm.x;
+          pw[e] = pr * (vmm.y * kappa);
+        }
+        const __half2 hi = __floats2half2_rn(pw[0], pw[1]);
+        const float2 hf = __half22float2(hi);
+        const __half2 lo = __floats2half2_rn(pw[0] - hf.x, pw[1] - hf.y);
+        xh[j][g2] = *reinterpret_cast<const uint32_t *>(&hi);
+        xl[j][g2] = *reinterpret_cast<const uint32_t *>(&lo);
       }
-      const __half2 hi = __floats2half2_rn(pw[0], pw[1]);
-      const float2 hf = __half22float2(hi);
-      const __half2 lo = __floats2half2_rn(pw[0] - hf.x, pw[1] - hf.y);
-      xh[g2] = *reinterpret_cast<const uint32_t *>(&hi);
-      xl[g2] = *reinterpret_cast<const uint32_t *>(&lo);
     }
-
-    // ---- values: O^T += C^T P' (codes and P' transposed in registers)
-    uint32_t vr0[KB][2], vr1[KB][2];
-    unpack_row<L>(sv + r * W, c, Lr, L2r, lut, vr0);
-    unpack_row<L>(sv + (8 + r) * W, c, Lr, L2r, lut, vr1);
+    // ---- B operands of the value MMAs: 8x8 matrices (rows = 8 tokens, columns
+    // 0..3 the hi parts and 4..7 the lo parts of the query heads), transposed
+    uint32_t bh[2][2], bl[2][2];          // [block][token r | r+8]
     if (pack_lo) {
-      // columns 0..3: hi parts (lanes c < 2), 4..7: lo parts (lanes c >= 2)
-      const uint32_t b0 = movmatrix_t(c < 2 ? xh[0] : xl[0]);
-      const uint32_t b1 = movmatrix_t(c < 2 ? xh[1] : xl[1]);
 #pragma unroll
-      for (int kb = 0; kb < KB; ++kb) {
-        const uint32_t a0 = movmatrix_t(vr0[kb][0]);
-        const uint32_t a1 = movmatrix_t(vr0[kb][1]);
-        const uint32_t a2 = movmatrix_t(vr1[kb][0]);
-        const uint32_t a3 = movmatrix_t(vr1[kb][1]);
-        mma_16816(oacc[kb], a0, a1, a2, a3, b0, b1);
+      for (int g2 = 0; g2 < 2; ++g2) {
+        // lane (r, c) supplies columns 2c, 2c+1: hi parts from the block-0 lane
+        // of its head pair, lo parts from the partner lane c^2
+        const uint32_t sxh = __shfl_xor_sync(0xffffffffu, xh[0][g2], 2);
+        const uint32_t sxl = __shfl_xor_sync(0xffffffffu, xl[0][g2], 2);
+        bh[0][g2] = movmatrix_t(c < 2 ? xh[0][g2] : sxl);
+        bh[1][g2] = movmatrix_t(c < 2 ? sxh : xl[0][g2]);
       }
     } else {
-      const uint32_t bh0 = movmatrix_t(xh[0]), bh1 = movmatrix_t(xh[1]);
-      const uint32_t bl0 = movmatrix_t(xl[0]), bl1 = movmatrix_t(xl[1]);
 #pragma unroll
-      for (int kb = 0; kb < KB; ++kb) {
-        const uint32_t a0 = movmatrix_t(vr0[kb][0]);
-        const uint32_t a1 = movmatrix_t(vr0[kb][1]);
-        const uint32_t a2 = movmatrix_t(vr1[kb][0]);
-        const uint32_t a3 = movmatrix_t(vr1[kb][1]);
-        mma_16816(oacc[kb], a0, a1, a2, a3, bh0, bh1);
-        mma_16816(oacc[kb], a0, a1, a2, a3, bl0, bl1);
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int g2 = 0; g2 < 2; ++g2) {
+          bh[j][g2] = movmatrix_t(xh[j][g2]);
+          bl[j][g2] = movmatrix_t(xl[j][g2]);
+        }
+    }
+
+    // ---- values: O^T += C^T P' (codes transposed in registers), word by word
+#pragma unroll
+    for (int i = 0; i < WPG; ++i) {
+#pragma unroll
+      for (int blk = 0; blk < 2; ++blk) {
+        uint32_t ra[RPW], rb[RPW];
+        unpack_word<L>(sv[(blk * 16 + r) * W + c * WPG + i], ra);
+        unpack_word<L>(sv[(blk * 16 + 8 + r) * W + c * WPG + i], rb);
+#pragma unroll
+        for (int m = 0; m < KPW; ++m) {
+          const int kb = i * KPW + m;
+          const uint32_t a0 = movmatrix_t(ra[2 * m]);
+          const uint32_t a1 = movmatrix_t(ra[2 * m + 1]);
+          const uint32_t a2 = movmatrix_t(rb[2 * m]);
+          const uint32_t a3 = movmatrix_t(rb[2 * m + 1]);
+          mma_16816(oacc[kb], a0, a1, a2, a3, bh[blk][0], bh[blk][1]);
+          if (!pack_lo) mma_16816(oacc[kb], a0, a1, a2, a3, bl[blk][0], bl[blk][1]);
+        }
       }
     }
     __syncwarp();
@@ -492,6 +589,12 @@ decode_pool_kernel(const DecParams p) {
       l_run[e] += __shfl_xor_sync(0xffffffffu, l_run[e], o);
       mt_run[e] += __shfl_xor_sync(0xffffffffu, mt_run[e], o);
     }
+  if (pack_lo)          // lanes c and c^2 took the two blocks of every tile, with the same running max
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      l_run[e] += __shfl_xor_sync(0xffffffffu, l_run[e], 2);
+      mt_run[e] += __shfl_xor_sync(0xffffffffu, mt_run[e], 2);
+    }
   if (pack_lo)
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb)
@@ -511,14 +614,16 @@ decode_pool_kernel(const DecParams p) {
         wst[(warp * DEC_GMAX + qc0 + e) * 3 + 1] = l_run[e];
         wst[(warp * DEC_GMAX + qc0 + e) * 3 + 2] = mt_run[e];
       }
-  constexpr float unscale = 16777216.0f / kappa;
+  constexpr float unscale = Gm::FAC / kappa;
   if (owner)
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         // slot r (hh=0) or 8+r (hh=1) of block kb belongs to lane group r/2, position (r%2) + 2hh
-        const int d = slot_dim<L>(r >> 1, 4 * kb + 2 * hh + (r & 1));
+        // (both candidate slots are compile-time, so the slot table folds away)
+        const int dA = slot_dim<L>(r >> 1, 4 * kb + 2 * hh), dB = slot_dim<L>(r >> 1, 4 * kb + 2 * hh + 1);
+        const int d = (r & 1) ? dB : dA;
         if (d >= 0) {
           if (qc0 < G) wo[(warp * DEC_GMAX + qc0) * kD + d] = oacc[kb][2 * hh] * unscale;
           if (qc0 + 1 < G) wo[(warp * DEC_GMAX + qc0 + 1) * kD + d] = oacc[kb][2 * hh + 1] * unscale;
@@ -526,7 +631,7 @@ decode_pool_kernel(const DecParams p) {
       }
     }
   __syncthreads();
-  float *dst = p.part + ((int64_t)slab * p.NU + p.unit0 + split) * G * PART_STRIDE;
+  float *dst = p.part + ((int64_t)slab * p.NU + pa.unit0 + split) * G * PART_STRIDE;
   for (int i = threadIdx.x; i < G * kD; i += DEC_WARPS * 32) {
     const int qh = i / kD, d = i % kD;
     float M = -INFINITY;
@@ -548,6 +653,24 @@ decode_pool_kernel(const DecParams p) {
       dst[qh * PART_STRIDE + 0] = M;
       dst[qh * PART_STRIDE + 1] = lsum;
     }
+  }
+}
+
+// Both pool classes in one launch (LA: class 0 = high, LB: class 1 = low), so
+// that the CTAs of the two pools fill the same waves; a launch with one class
+// uses LA == LB.
+template <int LA, int LB, bool ROT>
+__global__ void __launch_bounds__(DEC_WARPS * 32, 4) decode_pool_kernel(const DecParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int n0 = p.slabs * p.pool[0].S;
+  const int cls = (int)blockIdx.x >= n0;
+  const int i = cls ? (int)blockIdx.x - n0 : (int)blockIdx.x;
+  const int S = p.pool[cls].S;
+  if constexpr (LA == LB) {
+    pool_body<LA, ROT>(p, p.pool[cls], i / S, i % S, smem);
+  } else {
+    if (cls == 0) pool_body<LA, ROT>(p, p.pool[0], i / S, i % S, smem);
+    else pool_body<LB, ROT>(p, p.pool[1], i / S, i % S, smem);
   }
 }
 
@@ -709,63 +832,97 @@ __global__ void decode_score_acc_kernel(const float *__restrict__ prob, int H_q,
 // ---------------------------------------------------------------- host side
 template <int L>
 static int pool_smem_bytes(int G) {
-  return kQOff<L> + kLutBytes + kQfragBytes<L> + G * kD * 4;
+  return kQOff<L> + kQfragBytes<L> + G * kD * 4;
 }
 
-template <int L, bool ROT>
-static cudaError_t launch_pool(const DecParams &p, int grid, cudaStream_t st) {
-  const int smem = pool_smem_bytes<L>(p.G);
-  cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(decode_pool_kernel<L, ROT>),
-                                 pool_smem_bytes<L>(DEC_GMAX));
+template <int LA, int LB, bool ROT>
+static cudaError_t launch_pools(const DecParams &p, int grid, cudaStream_t st) {
+  const int smem = pool_smem_bytes<LA>(p.G) > pool_smem_bytes<LB>(p.G) ? pool_smem_bytes<LA>(p.G)
+                                                                        : pool_smem_bytes<LB>(p.G);
+  const int smax = pool_smem_bytes<LA>(DEC_GMAX) > pool_smem_bytes<LB>(DEC_GMAX) ? pool_smem_bytes<LA>(DEC_GMAX)
+                                                                                : pool_smem_bytes<LB>(DEC_GMAX);
+  cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT>), smax);
   if (e != cudaSuccess) return e;
-  decode_pool_kernel<L, ROT><<<grid, DEC_WARPS * 32, smem, st>>>(p);
+  if (grid > 0) decode_pool_kernel<LA, LB, ROT><<<grid, DEC_WARPS * 32, smem, st>>>(p);
   return cudaGetLastError();
 }
 
+// one class per launch, any level
 template <bool ROT>
-static cudaError_t launch_pool_rt(int L, const DecParams &p, int grid, cudaStream_t st) {
+static cudaError_t launch_one(int L, const DecParams &p, int grid, cudaStream_t st) {
   switch (L) {
-    case 2: return launch_pool<2, ROT>(p, grid, st);
-    case 3: return launch_pool<3, ROT>(p, grid, st);
-    case 4: return launch_pool<4, ROT>(p, grid, st);
-    case 5: return launch_pool<5, ROT>(p, grid, st);
-    case 6: return launch_pool<6, ROT>(p, grid, st);
-    case 7: return launch_pool<7, ROT>(p, grid, st);
-    case 8: return launch_pool<8, ROT>(p, grid, st);
-    case 9: return launch_pool<9, ROT>(p, grid, st);
-    case 10: return launch_pool<10, ROT>(p, grid, st);
-    case 11: return launch_pool<11, ROT>(p, grid, st);
-    case 12: return launch_pool<12, ROT>(p, grid, st);
-    case 13: return launch_pool<13, ROT>(p, grid, st);
-    case 14: return launch_pool<14, ROT>(p, grid, st);
-    case 15: return launch_pool<15, ROT>(p, grid, st);
-    case 16: return launch_pool<16, ROT>(p, grid, st);
+    case 2: return launch_pools<2, 2, ROT>(p, grid, st);
+    case 3: return launch_pools<3, 3, ROT>(p, grid, st);
+    case 4: return launch_pools<4, 4, ROT>(p, grid, st);
+    case 5: return launch_pools<5, 5, ROT>(p, grid, st);
+    case 6: return launch_pools<6, 6, ROT>(p, grid, st);
+    case 7: return launch_pools<7, 7, ROT>(p, grid, st);
+    case 8: return launch_pools<8, 8, ROT>(p, grid, st);
+    case 9: return launch_pools<9, 9, ROT>(p, grid, st);
+    case 10: return launch_pools<10, 10, ROT>(p, grid, st);
+    case 11: return launch_pools<11, 11, ROT>(p, grid, st);
+    case 12: return launch_pools<12, 12, ROT>(p, grid, st);
+    case 13: return launch_pools<13, 13, ROT>(p, grid, st);
+    case 14: return launch_pools<14, 14, ROT>(p, grid, st);
+    case 15: return launch_pools<15, 15, ROT>(p, grid, st);
+    case 16: return launch_pools<16, 16, ROT>(p, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-static cudaError_t launch_pool_any(int L, const DecParams &p, int grid, cudaStream_t st) {
-  return p.rot ? launch_pool_rt<true>(L, p, grid, st) : launch_pool_rt<false>(L, p, grid, st);
+// both classes in one launch: every uniform pair, and the adjacent pairs the
+// pages use (6/5) or sweep (5/4, 8/6, 16/8); other pairs take two launches
+static bool has_merged(int Lh, int Ll) {
+  return Lh == Ll || (Lh == 6 && Ll == 5) || (Lh == 5 && Ll == 4) || (Lh == 8 && Ll == 6) || (Lh == 16 && Ll == 8);
+}
+template <bool ROT>
+static cudaError_t launch_merged(int Lh, int Ll, const DecParams &p, int grid, cudaStream_t st) {
+  if (Lh == Ll) return launch_one<ROT>(Lh, p, grid, st);
+  if (Lh == 6 && Ll == 5) return launch_pools<6, 5, ROT>(p, grid, st);
+  if (Lh == 5 && Ll == 4) return launch_pools<5, 4, ROT>(p, grid, st);
+  if (Lh == 8 && Ll == 6) return launch_pools<8, 6, ROT>(p, grid, st);
+  return launch_pools<16, 8, ROT>(p, grid, st);
 }
 
-// splits per slab for a pool of capacity cap (host knows only capacities)
-static int pool_splits(const semkv_cache &c, int n_layers, int cap) {
-  const int sms = device_sm_count();
+// Splits per slab of each class (the host knows only capacities).  CTAs of
+// one launch run in rounds of R = 4 resident CTAs per SM; the model is
+//   time ~ rounds * (tiles of the longest CTA + a per-CTA overhead of 2 tiles)
+// with the splits of the two classes in proportion to their capacities, and
+// the smallest split count within 0.5% of the best is taken.  On the 32-layer
+// prefill cache (256 slabs, 1032 tiles per pool) this gives 8 splits per pool,
+// 4096 CTAs in 7 rounds of 592.
+static void pool_splits(const semkv_cache &c, int n_layers, int *Sh, int *Sl) {
+  const int64_t R = (int64_t)device_sm_count() * 4;
   const int64_t slabs = (int64_t)c.B * n_layers * c.H;
-  // about 1.75 waves of the 4 resident CTAs per SM, rounded to the nearest
-  // split count: on the 32-layer prefill cache (256 slabs) 4 splits took
-  // 0.584 ms against 0.666 (2), 0.675 (3), 0.616 (5), 0.627 (7), 0.614 (10)
-  const int64_t target = (int64_t)sms * 7;
-  int64_t S = (target + slabs / 2) / slabs;
-  const int64_t max_by_tiles = (cap / 16 + 15) / 16;  // keep >= 16 tiles (4 per warp) per unit
-  if (S > max_by_tiles) S = max_by_tiles;
-  if (S < 1) S = 1;
-  if (S > 64) S = 64;
-  return (int)S;
+  const int64_t th = (c.cap_high + 15) / 16, tl = (c.cap_low + 15) / 16;
+  const bool merged = has_merged(c.L_high, c.L_low);
+  const int64_t tmax = th > tl ? th : tl, tmin = th > tl ? tl : th;
+  double best = 1e300;
+  *Sh = *Sl = 1;
+  for (int S = 1; S <= 64; ++S) {
+    if (S > 1 && tmax / S < 16) break;                   // keep >= 16 tiles (4 per warp) per CTA
+    int s_small = tmax > 0 ? (int)((S * tmin + tmax / 2) / tmax) : 1;
+    if (s_small < 1) s_small = 1;
+    const int sh = th >= tl ? S : s_small, sl = th >= tl ? s_small : S;
+    const double wh = (double)th / sh + 2.0, wl = (double)tl / sl + 2.0;
+    double est;
+    if (merged) {
+      const int64_t rounds = (slabs * (sh + sl) + R - 1) / R;
+      est = rounds * (wh > wl ? wh : wl);
+    } else {
+      est = ((slabs * sh + R - 1) / R) * wh + ((slabs * sl + R - 1) / R) * wl;
+    }
+    if (est < best * 0.995) {
+      best = est;
+      *Sh = sh;
+      *Sl = sl;
+    }
+  }
 }
 
 size_t decode_ws_bytes(const semkv_cache &c, int n_layers) {
-  const int Sh = pool_splits(c, n_layers, c.cap_high), Sl = pool_splits(c, n_layers, c.cap_low);
+  int Sh, Sl;
+  pool_splits(c, n_layers, &Sh, &Sl);
   const int64_t slabs = (int64_t)c.B * n_layers * c.H;
   const int G = c.H_q / c.H;
   const size_t parts = (size_t)(slabs * (Sh + Sl + 1) * G * PART_STRIDE * sizeof(float));
@@ -774,11 +931,13 @@ size_t decode_ws_bytes(const semkv_cache &c, int n_layers) {
 
 cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int score_layer, const uint16_t *q,
                           uint16_t *out, float sm_scale, void *ws, uint32_t *status, cudaStream_t st) {
-  const int Sh = pool_splits(c, n_layers, c.cap_high), Sl = pool_splits(c, n_layers, c.cap_low);
+  int Sh, Sl;
+  pool_splits(c, n_layers, &Sh, &Sl);
   const int NU = Sh + Sl + 1;
   const int slabs = c.B * n_layers * c.H;
   const int G = c.H_q / c.H;
   DecParams p;
+  p.slabs = slabs;
   p.B = c.B;
   p.Lyr = c.n_layers;
   p.H = c.H;
@@ -791,23 +950,29 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int sc
   p.part = reinterpret_cast<float *>(ws);
   p.NU = NU;
   p.status = status;
-  p.wait0 = first_wait_polls(kWaitLimit);
-  cudaError_t e;
-  // high pool
-  p.kw = c.k_high; p.vw = c.v_high;
-  p.km = reinterpret_cast<const float2 *>(c.k_high_meta);
-  p.vm = reinterpret_cast<const float2 *>(c.v_high_meta);
-  p.count = c.n_high; p.cap = c.cap_high; p.unit0 = 0; p.S = Sh; p.Lrt = (uint32_t)c.L_high;
   p.rot = c.rotate;
-  e = launch_pool_any(c.L_high, p, slabs * Sh, st);
-  if (e != cudaSuccess) return e;
-  // low pool
-  p.kw = c.k_low; p.vw = c.v_low;
-  p.km = reinterpret_cast<const float2 *>(c.k_low_meta);
-  p.vm = reinterpret_cast<const float2 *>(c.v_low_meta);
-  p.count = c.n_low; p.cap = c.cap_low; p.unit0 = Sh; p.S = Sl; p.Lrt = (uint32_t)c.L_low;
-  e = launch_pool_any(c.L_low, p, slabs * Sl, st);
-  if (e != cudaSuccess) return e;
+  p.wait0 = first_wait_polls(kWaitLimit);
+  const PoolArgs high = {c.k_high, c.v_high, reinterpret_cast<const float2 *>(c.k_high_meta),
+                         reinterpret_cast<const float2 *>(c.v_high_meta), c.n_high, c.cap_high, Sh, 0};
+  const PoolArgs low = {c.k_low, c.v_low, reinterpret_cast<const float2 *>(c.k_low_meta),
+                        reinterpret_cast<const float2 *>(c.v_low_meta), c.n_low, c.cap_low, Sl, Sh};
+  cudaError_t e;
+  if (has_merged(c.L_high, c.L_low)) {
+    p.pool[0] = high;
+    p.pool[1] = low;
+    e = c.rotate ? launch_merged<true>(c.L_high, c.L_low, p, slabs * (Sh + Sl), st)
+                 : launch_merged<false>(c.L_high, c.L_low, p, slabs * (Sh + Sl), st);
+    if (e != cudaSuccess) return e;
+  } else {
+    for (int cls = 0; cls < 2; ++cls) {
+      p.pool[0] = cls ? low : high;
+      p.pool[1] = p.pool[0];
+      p.pool[1].S = 0;
+      const int L = cls ? c.L_low : c.L_high;
+      e = c.rotate ? launch_one<true>(L, p, slabs * p.pool[0].S, st) : launch_one<false>(L, p, slabs * p.pool[0].S, st);
+      if (e != cudaSuccess) return e;
+    }
+  }
   // FP16 block
   BufParams bp;
   bp.bk = c.buf_k; bp.bv = c.buf_v; bp.block = c.block; bp.buf_len = c.buf_len;

@@ -1,0 +1,85 @@
+"""The f16 digit-extraction constants of the decode kernel, checked exhaustively (CPU).
+
+decode.cu peels base-L digits off a part P of a packed word with
+    t = fma(X, c, K),  X = 1024 + P (first step) or 1536 + P (later steps),
+and relies on t == 1536 + floor(P / L) exactly for every part value the word
+layout can produce.  This test reads the (c, K) table from the kernel source
+and checks that property for every P, emulating the fused f16 multiply-add
+exactly: X, c and K are f16 values, so X*c + K is exact in float64 and one
+round-to-nearest-even to f16 is what the fused instruction does.  It also
+checks that the part sizes cover each word and that every part stays below
+1024, the range in which 1024 + P is an exact f16 integer.
+"""
+import os
+import re
+
+import numpy as np
+import pytest
+
+from oracle import semkv_oracle as O
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "kv_cache_mixed_b200", "csrc", "decode.cu")
+
+
+def _plans():
+    text = open(SRC).read()
+    rows = re.findall(r"L == (\d+)\s*\?\s*F16Plan\{(\d+), \{([\d, ]+)\}, (0x[0-9a-f]+), (0x[0-9a-f]+), "
+                      r"(0x[0-9a-f]+), (0x[0-9a-f]+)\}", text)
+    out = {}
+    for L, np_, parts, c0, k0, c1, k1 in rows:
+        p = [int(x) for x in parts.split(",")][:int(np_)]
+        out[int(L)] = (p, [int(v, 16) for v in (c0, k0, c1, k1)])
+    return out
+
+
+def _f16(bits):
+    return float(np.array([bits], dtype=np.uint16).view(np.float16)[0])
+
+
+def _step_ok(L, bias, pmax, c_bits, k_bits):
+    P = np.arange(pmax, dtype=np.float64)
+    exact = (bias + P) * _f16(c_bits) + _f16(k_bits)        # exact in float64 at these sizes
+    t = exact.astype(np.float16).astype(np.float64)         # one round-to-nearest-even to f16
+    return np.array_equal(t, 1536 + np.floor(P / L))
+
+
+def test_every_non_power_of_two_level_has_a_plan():
+    plans = _plans()
+    assert sorted(plans) == [L for L in range(3, 16) if L not in (4, 8)]
+
+
+@pytest.mark.parametrize("L", [L for L in range(3, 16) if L not in (4, 8)])
+def test_f16_steps_are_exact_for_every_part_value(L):
+    parts, (c0, k0, c1, k1) = _plans()[L]
+    assert sum(parts) == O.digits_per_word(L)            # the parts cover the word's digits
+    kmax = max(parts)
+    assert L ** kmax <= 1024                             # 1024 + P is an exact f16 integer
+    assert _step_ok(L, 1024, L ** kmax, c0, k0)          # first step of every register
+    if kmax > 1:
+        assert _step_ok(L, 1536, L ** (kmax - 1), c1, k1)   # every later step
+    # the quotient of a pair register by multiply-high is exact: L^ka * L^(ka+kb) < 2^32
+    for j in range(0, len(parts), 2):
+        ka = parts[j]
+        kb = parts[j + 1] if j + 1 < len(parts) else 0
+        assert L ** ka * L ** (ka + kb) < 2 ** 32
+
+
+@pytest.mark.parametrize("L", [L for L in range(3, 16) if L not in (4, 8)])
+def test_digit_chain_reproduces_base_L_digits(L):
+    """The whole f16 chain on one part, emulated step by step, gives the digits."""
+    parts, (c0, k0, c1, k1) = _plans()[L]
+    k = max(parts)
+    P = np.arange(L ** k, dtype=np.float64)
+    X = 1024 + P
+    c, K, bias = _f16(c0), _f16(k0), 1024.0
+    digits = []
+    for s in range(k - 1):
+        t = (X * c + K).astype(np.float16).astype(np.float64)
+        sp = (t * -L + (1536 * L - bias)).astype(np.float16).astype(np.float64)
+        digits.append((X + sp).astype(np.float16).astype(np.float64))
+        X, c, K, bias = t, _f16(c1), _f16(k1), 1536.0
+    digits.append((X - 1536.0 if k > 1 else X - 1024.0))
+    ref = [(np.arange(L ** k) // L ** s) % L for s in range(k)]
+    for s in range(k):
+        assert np.array_equal(digits[s], ref[s]), (L, s)

@@ -80,7 +80,9 @@ def test_llama8b_prefill_full_size():
     s_ref = O.score_attn_mass(to_np(k[0, Lyr - 1]), to_np(q_win[0]), T)
     assert np.all(np.abs(to_np(score)[0] - s_ref) <= SCORE_RTOL * np.abs(s_ref) + SCORE_ATOL)
     m = O.select_mask(s_ref.astype(np.float32), nh)
-    check_mask_near_threshold(to_np(mask)[0], s_ref, m, nh)
+    flips = check_mask_near_threshold(to_np(mask)[0], s_ref, m, nh)
+    print(f"[mask flips] {wl.name} seq 0: {flips} of {T} tokens differ from the oracle's mask, "
+          f"all within the score tolerance of the threshold")
 
     # quantize + decode of the whole cache, on the oracle's mask
     mask.copy_(torch.from_numpy(m)[None])
@@ -164,7 +166,9 @@ def test_level_sweep_full_size(L_high, L_low):
         s_ref = O.score_attn_mass(to_np(k[b, 0]), to_np(q_win[b]), T)
         assert np.all(np.abs(to_np(score)[b] - s_ref) <= SCORE_RTOL * np.abs(s_ref) + SCORE_ATOL)
         m_all[b] = O.select_mask(s_ref.astype(np.float32), nh)
-        check_mask_near_threshold(to_np(mask)[b], s_ref, m_all[b], nh)
+        flips = check_mask_near_threshold(to_np(mask)[b], s_ref, m_all[b], nh)
+        print(f"[mask flips] {wl.name} {L_high}/{L_low} seq {b}: {flips} of {T} tokens differ from the "
+              f"oracle's mask, all within the score tolerance of the threshold")
     mask.copy_(torch.from_numpy(m_all))
     cache = _cache_for(kv, wl, wl.r_ppm, T, L_high, L_low)
     kv.semkv_quantize(cache, k, v, seq_len, mask)
@@ -211,7 +215,9 @@ def test_generation_full_size():
         s_ref = O.score_attn_mass(to_np(k[b, Lyr - 1]), to_np(q_win[b]), T0)
         nh = O.num_high(T0, wl.r_ppm)
         m_all[b, :T0] = O.select_mask(s_ref.astype(np.float32), nh)
-        check_mask_near_threshold(to_np(mask)[b, :T0], s_ref, m_all[b, :T0], nh)
+        flips = check_mask_near_threshold(to_np(mask)[b, :T0], s_ref, m_all[b, :T0], nh)
+        print(f"[mask flips] {wl.name} seq {b}: {flips} of {T0} tokens differ from the oracle's mask, "
+              f"all within the score tolerance of the threshold")
     mask.copy_(torch.from_numpy(m_all))
     cache = _cache_for(kv, wl, wl.r_ppm, T, gen=wl.gen_steps)
     kv.semkv_quantize(cache, k, v, seq_len, mask)
