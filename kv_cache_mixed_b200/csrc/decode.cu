@@ -847,6 +847,47 @@ static cudaError_t launch_pools(const DecParams &p, int grid, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// resident CTAs per SM of the kernel instance <LA, LB, ROT> (queried once per device)
+template <int LA, int LB, bool ROT>
+static int pools_occupancy(int G) {
+  const int smem = pool_smem_bytes<LA>(G) > pool_smem_bytes<LB>(G) ? pool_smem_bytes<LA>(G) : pool_smem_bytes<LB>(G);
+  const int smax = pool_smem_bytes<LA>(DEC_GMAX) > pool_smem_bytes<LB>(DEC_GMAX) ? pool_smem_bytes<LA>(DEC_GMAX)
+                                                                                : pool_smem_bytes<LB>(DEC_GMAX);
+  const void *fn = reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT>);
+  int nb = 1;
+  if (prepare_kernel(fn, smax) != cudaSuccess || kernel_occupancy(fn, DEC_WARPS * 32, smem, &nb) != cudaSuccess)
+    return 1;
+  return nb;
+}
+template <bool ROT>
+static int occupancy_one(int L, int G) {
+  switch (L) {
+    case 2: return pools_occupancy<2, 2, ROT>(G);
+    case 3: return pools_occupancy<3, 3, ROT>(G);
+    case 4: return pools_occupancy<4, 4, ROT>(G);
+    case 5: return pools_occupancy<5, 5, ROT>(G);
+    case 6: return pools_occupancy<6, 6, ROT>(G);
+    case 7: return pools_occupancy<7, 7, ROT>(G);
+    case 8: return pools_occupancy<8, 8, ROT>(G);
+    case 9: return pools_occupancy<9, 9, ROT>(G);
+    case 10: return pools_occupancy<10, 10, ROT>(G);
+    case 11: return pools_occupancy<11, 11, ROT>(G);
+    case 12: return pools_occupancy<12, 12, ROT>(G);
+    case 13: return pools_occupancy<13, 13, ROT>(G);
+    case 14: return pools_occupancy<14, 14, ROT>(G);
+    case 15: return pools_occupancy<15, 15, ROT>(G);
+    default: return pools_occupancy<16, 16, ROT>(G);
+  }
+}
+template <bool ROT>
+static int occupancy_merged(int Lh, int Ll, int G) {
+  if (Lh == Ll) return occupancy_one<ROT>(Lh, G);
+  if (Lh == 6 && Ll == 5) return pools_occupancy<6, 5, ROT>(G);
+  if (Lh == 5 && Ll == 4) return pools_occupancy<5, 4, ROT>(G);
+  if (Lh == 8 && Ll == 6) return pools_occupancy<8, 6, ROT>(G);
+  return pools_occupancy<16, 8, ROT>(G);
+}
+
 // one class per launch, any level
 template <bool ROT>
 static cudaError_t launch_one(int L, const DecParams &p, int grid, cudaStream_t st) {
@@ -885,17 +926,26 @@ static cudaError_t launch_merged(int Lh, int Ll, const DecParams &p, int grid, c
 }
 
 // Splits per slab of each class (the host knows only capacities).  CTAs of
-// one launch run in rounds of R = 4 resident CTAs per SM; the model is
+// one launch run in rounds of R = resident CTAs per SM x SMs; the model is
 //   time ~ rounds * (tiles of the longest CTA + a per-CTA overhead of 2 tiles)
 // with the splits of the two classes in proportion to their capacities, and
 // the smallest split count within 0.5% of the best is taken.  On the 32-layer
-// prefill cache (256 slabs, 1032 tiles per pool) this gives 8 splits per pool,
-// 4096 CTAs in 7 rounds of 592.
+// prefill cache (256 slabs, 1032 16-token tiles per pool, 4 CTAs per SM) this
+// gives 8 splits per pool, 4096 CTAs in 7 rounds of 592.
 static void pool_splits(const semkv_cache &c, int n_layers, int *Sh, int *Sl) {
-  const int64_t R = (int64_t)device_sm_count() * 4;
+  const bool merged = has_merged(c.L_high, c.L_low);
+  const int G = c.H_q / c.H;
+  int occ;
+  if (merged) {
+    occ = c.rotate ? occupancy_merged<true>(c.L_high, c.L_low, G) : occupancy_merged<false>(c.L_high, c.L_low, G);
+  } else {
+    const int oh = c.rotate ? occupancy_one<true>(c.L_high, G) : occupancy_one<false>(c.L_high, G);
+    const int ol = c.rotate ? occupancy_one<true>(c.L_low, G) : occupancy_one<false>(c.L_low, G);
+    occ = oh < ol ? oh : ol;
+  }
+  const int64_t R = (int64_t)device_sm_count() * occ;
   const int64_t slabs = (int64_t)c.B * n_layers * c.H;
   const int64_t th = (c.cap_high + 15) / 16, tl = (c.cap_low + 15) / 16;
-  const bool merged = has_merged(c.L_high, c.L_low);
   const int64_t tmax = th > tl ? th : tl, tmin = th > tl ? tl : th;
   double best = 1e300;
   *Sh = *Sl = 1;

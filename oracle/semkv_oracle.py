@@ -23,6 +23,7 @@ cases, and the compression figures the pages print (tests/golden/).
 from __future__ import annotations
 
 import math
+from fractions import Fraction
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -501,3 +502,94 @@ def pages_effective_bits(levels_and_fracs, meta_scalars: int, D: int = HEAD_DIM)
 def layout_bytes_per_row(L: int, D: int = HEAD_DIM) -> int:
     """Bytes of one row in the library's layout: 32-bit mixed-radix words + fp32 (mn, scale)."""
     return 4 * words_per_row(L, D) + 8
+
+
+# ---------------------------------------------------------------------------
+# f1: the pages' own storage layout (SemKV, Table 3, Table 5, Table 6, Fig. 11:
+# "effective bits include packing and per-row metadata", two 16-bit scalars)
+# ---------------------------------------------------------------------------
+def pages_group(L: int, max_group: int = 5):
+    """(g, b) of the pages' packing: g <= 5 base-L digits held in b whole bits,
+    b the fewest bits that hold L**g values, with the g of fewest bits per digit
+    (of equal ones, the largest g).  Reading of the printed code bits
+    (pages_code_bits): 5 levels -> 3 digits in 7 bits, 6 levels -> 5 in 13."""
+    best = None
+    for k in range(1, max_group + 1):
+        b = (L ** k - 1).bit_length()
+        key = (Fraction(b, k), -k)
+        if best is None or key < best[0]:
+            best = (key, k, b)
+    return best[1], best[2]
+
+
+def pages_row_bits(L: int, D: int = HEAD_DIM) -> int:
+    """Code bits of one row: D // g full groups of b bits, then a tail group of
+    the D % g remaining digits in the fewest bits that hold L**(D % g) values."""
+    g, b = pages_group(L)
+    t = D % g
+    return (D // g) * b + ((L ** t - 1).bit_length() if t else 0)
+
+
+def pages_groups(L: int, D: int = HEAD_DIM):
+    """[(first digit, digits, bits, bit offset in the row)] of every group of a row."""
+    g, b = pages_group(L)
+    out, off, d0 = [], 0, 0
+    while d0 < D:
+        k = min(g, D - d0)
+        bits = (L ** k - 1).bit_length()
+        out.append((d0, k, bits, off))
+        off += bits
+        d0 += k
+    return out
+
+
+def pack_rows_pages(codes: np.ndarray, L: int) -> np.ndarray:
+    """Rows of codes uint8 [n][D] -> the pages' bit stream, uint8 bytes.
+
+    Row s occupies stream bits [s*R, (s+1)*R), R = pages_row_bits(L): rows sit
+    back to back at bit granularity (reading: no padding, so that the stored
+    bytes are the printed effective bits).  Stream bit k is bit k % 8 of byte
+    k // 8.  Group (d0, k, bits, off) of a row holds the value
+    sum_j codes[d0 + j] * L**j (digit 0 least significant) in row bits
+    [off, off + bits), least significant bit first.  The stream is zero-padded
+    to whole bytes.
+    """
+    n, D = codes.shape
+    R = pages_row_bits(L, D)
+    stream = np.zeros(n * R, dtype=np.uint8)
+    rows = np.arange(n, dtype=np.int64) * R
+    for d0, k, bits, off in pages_groups(L, D):
+        val = np.zeros(n, dtype=np.int64)
+        for j in reversed(range(k)):
+            val = val * L + codes[:, d0 + j].astype(np.int64)
+        for i in range(bits):
+            stream[rows + off + i] = (val >> i) & 1
+    return np.packbits(stream, bitorder="little")
+
+
+def unpack_rows_pages(stream: np.ndarray, n: int, L: int, D: int = HEAD_DIM) -> np.ndarray:
+    """Inverse of pack_rows_pages: uint8 codes [n][D], by repeated division of each group."""
+    bits = np.unpackbits(np.asarray(stream, dtype=np.uint8), bitorder="little")
+    R = pages_row_bits(L, D)
+    rows = np.arange(n, dtype=np.int64) * R
+    codes = np.zeros((n, D), dtype=np.uint8)
+    for d0, k, nb, off in pages_groups(L, D):
+        val = np.zeros(n, dtype=np.int64)
+        for i in range(nb):
+            val |= bits[rows + off + i].astype(np.int64) << i
+        for j in range(k):
+            codes[:, d0 + j] = val % L
+            val //= L
+    return codes
+
+
+def pages_meta(mn: np.ndarray, scale: np.ndarray):
+    """The two 16-bit scalars of a row: (min, scale) rounded to float16, nearest-even.
+    A scale that does not fit float16 (possible only for L = 2) becomes inf."""
+    with np.errstate(over="ignore"):
+        return mn.astype(np.float16), scale.astype(np.float16)
+
+
+def pages_layout_bytes(n_rows: int, L: int, D: int = HEAD_DIM) -> int:
+    """Bytes of n_rows rows in the pages' layout: the bit stream plus 4 bytes of scalars per row."""
+    return (n_rows * pages_row_bits(L, D) + 7) // 8 + 4 * n_rows
