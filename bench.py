@@ -400,9 +400,28 @@ def run_extensions(state, reps=5):
     rq_ms = med(rq)
     rd_ms = med(lambda: kv.semkv_decode_attn(rc, 0, Lyr, qdec, out))
     assert rc.status_flags() == 0 and cache.status_flags() == 0
+    del rc
+    # the pages' own storage layout (groups of <= 5 digits in whole bits, rows
+    # back to back in one bit stream, fp16 scalars)
+    pc = kv.MixedCache(B, Lyr, H, H_q, wl.L_high, wl.L_low, wl.r_ppm, nh + 128, T - nh + 128,
+                       layout=kv.LAYOUT_PAGES)
+
+    def pq():
+        pc.n_high.zero_()
+        pc.n_low.zero_()
+        kv.semkv_quantize(pc, k, v, seq_len, mask)
+    pq_ms = med(pq)
+    pd_ms = med(lambda: kv.semkv_decode_attn(pc, 0, Lyr, qdec, out))
+    assert pc.status_flags() == 0
+    pbytes = pc.pool_bytes()
     return {"decode_acc_ms": round(acc_ms, 4),
             "rotated": {"quantize_ms": round(rq_ms, 4), "decode_ms": round(rd_ms, 4),
-                        "quantize_gbs_fp16_in": round(fp16_in / (rq_ms * 1e-3) / 1e9, 1)}}
+                        "quantize_gbs_fp16_in": round(fp16_in / (rq_ms * 1e-3) / 1e9, 1)},
+            "pages_layout": {"quantize_ms": round(pq_ms, 4), "decode_ms": round(pd_ms, 4),
+                             "quantize_gbs_fp16_in": round(fp16_in / (pq_ms * 1e-3) / 1e9, 1),
+                             "decode_gbs_cache_read": round(pbytes / (pd_ms * 1e-3) / 1e9, 1),
+                             "pool_bytes": pbytes, "compression_vs_fp16": round(fp16_in / pbytes, 3),
+                             "row_bits_high_low": [pc.row_bits_high, pc.row_bits_low]}}
 
 
 def run_e2e(args, state, dist=None):

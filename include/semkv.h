@@ -42,7 +42,7 @@ extern "C" {
 typedef enum semkv_status {
   SEMKV_OK = 0,
   SEMKV_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape    */
-  SEMKV_ERR_UNSUPPORTED = 2,   /* D != 128, L outside [2,16], H_q/H > 8 (> 4 with rotate) */
+  SEMKV_ERR_UNSUPPORTED = 2,   /* D != 128, L outside [2,16], H_q/H > 8 (> 4 with rotate), a level the layout lacks */
   SEMKV_ERR_WORKSPACE = 3,     /* workspace smaller than the *_workspace_size    */
   SEMKV_ERR_CAPACITY = 4,      /* an append would overflow the FP16 block        */
   SEMKV_ERR_CUDA = 5           /* a launch failed (cudaGetLastError)             */
@@ -60,6 +60,11 @@ typedef enum semkv_score_kind {
 } semkv_score_kind;
 
 #define SEMKV_FLUSH 0x1u       /* semkv_append_block: quantize the partial FP16 block (end of turn, Fig. 6) */
+
+/* Pool storage layouts (semkv_cache.layout) */
+#define SEMKV_LAYOUT_WORDS 0   /* floor(32/log2 L) base-L digits per 32-bit word, fp32 (min, scale) */
+#define SEMKV_LAYOUT_PAGES 1   /* groups of <= 5 digits in whole bits, rows back to back in a bit
+                                  stream, fp16 (min, scale): the layout of Table 3/5/6, Fig. 11 */
 
 /*
  * The mixed cache.  A host-side struct of sizes and device pointers; the pools
@@ -81,6 +86,24 @@ typedef enum semkv_score_kind {
  * is quantized and stored, (min, scale) are x''s.  Decode rotates q the same
  * way and returns H o' / 128, so outputs are in the tokens' own basis.  The
  * FP16 block is stored unrotated.  Needs H_q/H <= 4 (UNSUPPORTED otherwise).
+ *
+ * layout = SEMKV_LAYOUT_PAGES (SemKV, Table 3, Table 5, Table 6, Fig. 11: the
+ * printed effective bits "include packing and per-row metadata" -- groups of
+ * at most five base-L digits in whole bits and two 16-bit scalars per row):
+ *   - a row's D codes form groups of g digits (the last group holds D mod g),
+ *     g and the group's bit width b chosen as semkv_row_bits documents; group
+ *     value = sum_j code[j] L^j (digit 0 least significant), least significant
+ *     bit first; a row is R = semkv_row_bits(1, L) bits;
+ *   - codes k_c, v_c: per (sequence, layer, head) slab one little-endian bit
+ *     stream of semkv_pool_words(1, L_c, cap_c) uint32 words, row s at bits
+ *     [s R, (s+1) R): rows sit back to back with no padding, so the stored
+ *     bytes are the printed effective bits;
+ *   - meta k_c_meta, v_c_meta: per row one 4-byte record of two IEEE fp16
+ *     values (min, scale), [B][n_layers][H][cap_c], the fp32 min and scale
+ *     rounded to nearest-even (the codes are those of the fp32 scalars);
+ *   - levels 9, 12, 14 and 15 are UNSUPPORTED, and so is rotate = 1.
+ * Quantize writes a row's boundary words with atomic bit operations, so rows
+ * of one slab may be written concurrently and no zero-filling is needed.
  */
 typedef struct semkv_cache {
   int32_t B, n_layers, H, H_q, D;
@@ -90,6 +113,7 @@ typedef struct semkv_cache {
   int32_t block;                 /* FP16 block length (128)                          */
   int32_t buf_len;               /* host: tokens in the FP16 block, 0 <= buf_len < block */
   int32_t rotate;                /* 0, or 1: Hadamard-rotated rows (Table 2), see below */
+  int32_t layout;                /* SEMKV_LAYOUT_WORDS (0) or SEMKV_LAYOUT_PAGES (1), see below */
   uint32_t *k_high, *v_high, *k_low, *v_low;
   float *k_high_meta, *v_high_meta, *k_low_meta, *v_low_meta;
   int32_t *n_high, *n_low;       /* device [B] */
@@ -109,6 +133,20 @@ int32_t semkv_digits_per_word(int32_t L);
 
 /* 32-bit words per row of D codes: ceil(D / digits_per_word(L)); -1 if invalid. */
 int32_t semkv_words_per_row(int32_t L, int32_t D);
+
+/* Code bits of one 128-value row in a layout: 32 * semkv_words_per_row(L, 128)
+ * for SEMKV_LAYOUT_WORDS; for SEMKV_LAYOUT_PAGES, g <= 5 digits per group in b
+ * bits, b the fewest bits holding L^g values and g the choice with the fewest
+ * bits per digit (the largest g among equals), plus the last group's
+ * 128 mod g digits in the fewest bits holding them (6 levels: 5 digits in 13
+ * bits, 333 bits a row; 5 levels: 3 digits in 7 bits, 299 bits a row).
+ * -1 for an invalid or unsupported (layout, L). */
+int32_t semkv_row_bits(int32_t layout, int32_t L);
+
+/* uint32 words of codes that one (sequence, layer, head) slab of a pool class
+ * of capacity cap occupies: cap * words_per_row for SEMKV_LAYOUT_WORDS,
+ * ceil(cap * row_bits / 128) * 4 for SEMKV_LAYOUT_PAGES.  -1 if invalid. */
+int64_t semkv_pool_words(int32_t layout, int32_t L, int32_t cap);
 
 /* Library build identification string (static storage). */
 const char *semkv_version(void);

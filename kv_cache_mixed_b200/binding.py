@@ -25,6 +25,7 @@ STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED", 3: "ERR_WOR
 FLAG_NONFINITE, FLAG_CAPACITY, FLAG_SEQLEN, FLAG_TIMEOUT = 0x1, 0x2, 0x4, 0x8
 SCORE_ATTN_MASS, SCORE_KEY_L2 = 0, 1
 FLUSH = 0x1
+LAYOUT_WORDS, LAYOUT_PAGES = 0, 1
 
 _p = ctypes.c_void_p
 _i32, _i64, _u32, _sz, _f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_size_t, ctypes.c_float
@@ -33,7 +34,7 @@ _i32, _i64, _u32, _sz, _f32 = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, c
 class SemkvCache(ctypes.Structure):
     """Mirror of struct semkv_cache."""
     _fields_ = [(n, _i32) for n in ("B", "n_layers", "H", "H_q", "D", "L_high", "L_low", "r_ppm",
-                                     "cap_high", "cap_low", "block", "buf_len", "rotate")] + \
+                                     "cap_high", "cap_low", "block", "buf_len", "rotate", "layout")] + \
                [(n, _p) for n in ("k_high", "v_high", "k_low", "v_low", "k_high_meta", "v_high_meta",
                                   "k_low_meta", "v_low_meta", "n_high", "n_low", "buf_k", "buf_v",
                                   "buf_score")]
@@ -49,6 +50,8 @@ def _sig(name, res, args):
 _lib_num_high = _sig("semkv_num_high", _i64, [_i64, _i32])
 _lib_digits = _sig("semkv_digits_per_word", _i32, [_i32])
 _lib_words = _sig("semkv_words_per_row", _i32, [_i32, _i32])
+_lib_row_bits = _sig("semkv_row_bits", _i32, [_i32, _i32])
+_lib_pool_words = _sig("semkv_pool_words", _i64, [_i32, _i32, _i32])
 _lib_version = _sig("semkv_version", ctypes.c_char_p, [])
 _lib_set_wait0 = _sig("semkv_set_first_copy_wait_polls", None, [_i32])
 _lib_score_ws = _sig("semkv_score_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32, _i32])
@@ -69,7 +72,8 @@ _lib_decode = _sig("semkv_decode_attn", _i32, [ctypes.POINTER(SemkvCache), _i32,
 _lib_decode_acc = _sig("semkv_decode_attn_acc", _i32, [ctypes.POINTER(SemkvCache), _i32, _i32, _i32, _p, _p, _f32,
                                                       _p, _sz, _p, _p])
 
-EXPORTED = ["semkv_num_high", "semkv_digits_per_word", "semkv_words_per_row", "semkv_version",
+EXPORTED = ["semkv_num_high", "semkv_digits_per_word", "semkv_words_per_row", "semkv_row_bits",
+            "semkv_pool_words", "semkv_version",
             "semkv_set_first_copy_wait_polls",
             "semkv_score_workspace_size", "semkv_score", "semkv_select_workspace_size", "semkv_select",
             "semkv_quantize_workspace_size", "semkv_quantize", "semkv_quantize_noalloc",
@@ -112,6 +116,14 @@ def semkv_words_per_row(L: int, D: int = 128) -> int:
     return int(_lib_words(L, D))
 
 
+def semkv_row_bits(layout: int, L: int) -> int:
+    return int(_lib_row_bits(layout, L))
+
+
+def semkv_pool_words(layout: int, L: int, cap: int) -> int:
+    return int(_lib_pool_words(layout, L, cap))
+
+
 def semkv_version() -> str:
     return _lib_version().decode()
 
@@ -148,24 +160,41 @@ def semkv_select(score: torch.Tensor, seq_len, r_ppm: int, mask: torch.Tensor, l
 class MixedCache:
     """Device memory of one mixed cache (pools, counts, FP16 block) and its C struct.
 
-    Pools are torch tensors on `device`, laid out as include/semkv.h describes.
+    Pools are torch tensors on `device`, laid out as include/semkv.h describes:
+    with layout=LAYOUT_WORDS the codes are int32 [B][n_layers][H][cap][W] and the
+    meta float32 [B][n_layers][H][cap][2]; with layout=LAYOUT_PAGES the codes are
+    one int32 bit stream [B][n_layers][H][semkv_pool_words(...)] per slab and the
+    meta float16 [B][n_layers][H][cap][2].
     """
 
     def __init__(self, B, n_layers, H, H_q, L_high, L_low, r_ppm, cap_high, cap_low, block=128,
-                 device="cuda", rotate=False):
+                 device="cuda", rotate=False, layout=LAYOUT_WORDS):
         self.device = torch.device(device)
         cap_high = (int(cap_high) + 15) // 16 * 16
         cap_low = (int(cap_low) + 15) // 16 * 16
+        self.layout = layout
         self.W_high = semkv_words_per_row(L_high)
         self.W_low = semkv_words_per_row(L_low)
+        self.row_bits_high = semkv_row_bits(layout, L_high)
+        self.row_bits_low = semkv_row_bits(layout, L_low)
+        if self.row_bits_high < 0 or self.row_bits_low < 0:
+            raise SemkvError("semkv_row_bits: ERR_UNSUPPORTED (level not available in this layout)")
         d = self.device
-        self.k_high = torch.zeros((B, n_layers, H, cap_high, self.W_high), dtype=torch.int32, device=d)
+        if layout == LAYOUT_PAGES:
+            def codes(L, cap):
+                return torch.zeros((B, n_layers, H, semkv_pool_words(layout, L, cap)), dtype=torch.int32, device=d)
+            mdt = torch.float16
+        else:
+            def codes(L, cap):
+                return torch.zeros((B, n_layers, H, cap, semkv_words_per_row(L)), dtype=torch.int32, device=d)
+            mdt = torch.float32
+        self.k_high = codes(L_high, cap_high)
         self.v_high = torch.zeros_like(self.k_high)
-        self.k_low = torch.zeros((B, n_layers, H, cap_low, self.W_low), dtype=torch.int32, device=d)
+        self.k_low = codes(L_low, cap_low)
         self.v_low = torch.zeros_like(self.k_low)
-        self.k_high_meta = torch.zeros((B, n_layers, H, cap_high, 2), dtype=torch.float32, device=d)
+        self.k_high_meta = torch.zeros((B, n_layers, H, cap_high, 2), dtype=mdt, device=d)
         self.v_high_meta = torch.zeros_like(self.k_high_meta)
-        self.k_low_meta = torch.zeros((B, n_layers, H, cap_low, 2), dtype=torch.float32, device=d)
+        self.k_low_meta = torch.zeros((B, n_layers, H, cap_low, 2), dtype=mdt, device=d)
         self.v_low_meta = torch.zeros_like(self.k_low_meta)
         self.n_high = torch.zeros(B, dtype=torch.int32, device=d)
         self.n_low = torch.zeros(B, dtype=torch.int32, device=d)
@@ -174,7 +203,7 @@ class MixedCache:
         self.buf_score = torch.zeros((B, block), dtype=torch.float32, device=d)
         self.status = torch.zeros(1, dtype=torch.int32, device=d)
         self.c = SemkvCache(B, n_layers, H, H_q, 128, L_high, L_low, r_ppm, cap_high, cap_low, block, 0,
-                            1 if rotate else 0,
+                            1 if rotate else 0, int(layout),
                             *[t.data_ptr() for t in (self.k_high, self.v_high, self.k_low, self.v_low,
                                                      self.k_high_meta, self.v_high_meta, self.k_low_meta,
                                                      self.v_low_meta, self.n_high, self.n_low, self.buf_k,
@@ -203,6 +232,8 @@ class MixedCache:
         nh = self.n_high.sum().item()
         nl = self.n_low.sum().item()
         rows = self.c.n_layers * self.c.H * 2
+        if self.layout == LAYOUT_PAGES:
+            return int(rows * ((nh * self.row_bits_high + 7) // 8 + (nl * self.row_bits_low + 7) // 8 + 4 * (nh + nl)))
         return int(rows * (nh * (4 * self.W_high + 8) + nl * (4 * self.W_low + 8)))
 
 

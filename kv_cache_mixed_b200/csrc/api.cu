@@ -34,6 +34,10 @@ semkv_status check_cache(const semkv_cache *c) {
   if (c->block < 1 || c->block > 128) return SEMKV_ERR_INVALID_ARG;
   if (c->rotate != 0 && c->rotate != 1) return SEMKV_ERR_INVALID_ARG;
   if (c->rotate && c->H_q / c->H > 4) return SEMKV_ERR_UNSUPPORTED;
+  if (c->layout != SEMKV_LAYOUT_WORDS && c->layout != SEMKV_LAYOUT_PAGES) return SEMKV_ERR_INVALID_ARG;
+  if (c->layout == SEMKV_LAYOUT_PAGES &&
+      (c->rotate || !pages_supported(c->L_high) || !pages_supported(c->L_low)))
+    return SEMKV_ERR_UNSUPPORTED;
   if (c->buf_len < 0 || c->buf_len >= c->block) return SEMKV_ERR_INVALID_ARG;
   const void *ptrs[] = {c->k_high, c->v_high, c->k_low, c->v_low, c->k_high_meta, c->v_high_meta,
                         c->k_low_meta, c->v_low_meta, c->n_high, c->n_low, c->buf_k, c->buf_v,
@@ -85,6 +89,7 @@ semkv_status quantize_rows(semkv_cache *c, const uint16_t *k, const uint16_t *v,
   q.cap_low = c->cap_low;
   q.L_high = c->L_high;
   q.rotate = c->rotate;
+  q.layout = c->layout;
   q.L_low = c->L_low;
   q.status = status;
   return cuda_status(launch_quantize(q, st));
@@ -130,7 +135,21 @@ int32_t semkv_words_per_row(int32_t L, int32_t D) {
   return (D + n - 1) / n;
 }
 
-const char *semkv_version(void) { return "semkv-b200 0.2 (sm_100a)"; }
+int32_t semkv_row_bits(int32_t layout, int32_t L) {
+  if (L < 2 || L > kMaxL) return -1;
+  if (layout == SEMKV_LAYOUT_WORDS) return 32 * words_per_row(L);
+  if (layout == SEMKV_LAYOUT_PAGES) return pages_supported(L) ? pages_row_bits(L) : -1;
+  return -1;
+}
+
+int64_t semkv_pool_words(int32_t layout, int32_t L, int32_t cap) {
+  const int32_t R = semkv_row_bits(layout, L);
+  if (R < 0 || cap < 0) return -1;
+  if (layout == SEMKV_LAYOUT_WORDS) return (int64_t)cap * words_per_row(L);
+  return ((int64_t)cap * R + 127) / 128 * 4;
+}
+
+const char *semkv_version(void) { return "semkv-b200 0.3 (sm_100a)"; }
 
 void semkv_set_first_copy_wait_polls(int32_t polls) { g_first_wait_polls = polls < 0 ? -1 : polls; }
 

@@ -35,6 +35,41 @@ __host__ __device__ constexpr unsigned long long ipow(int L, int k) {
 }
 
 // ---------------------------------------------------------------------------
+// The pages' layout (SEMKV_LAYOUT_PAGES): groups of g <= 5 digits in b bits
+// ---------------------------------------------------------------------------
+// fewest bits that hold n values
+__host__ __device__ constexpr int bits_for(unsigned long long n) {
+  int b = 0;
+  while ((1ull << b) < n) ++b;
+  return b;
+}
+// g: the group size with the fewest bits per digit, the largest among equals
+__host__ __device__ constexpr int pages_g(int L) {
+  int best_k = 1, best_b = bits_for(ipow(L, 1));
+  for (int k = 2; k <= 5; ++k) {
+    const int b = bits_for(ipow(L, k));
+    if (b * best_k <= best_b * k) {        // b/k <= best_b/best_k
+      best_k = k;
+      best_b = b;
+    }
+  }
+  return best_k;
+}
+__host__ __device__ constexpr int pages_b(int L) { return bits_for(ipow(L, pages_g(L))); }
+__host__ __device__ constexpr int pages_tail(int L) { return kD % pages_g(L); }
+__host__ __device__ constexpr int pages_groups(int L) { return (kD + pages_g(L) - 1) / pages_g(L); }
+__host__ __device__ constexpr int pages_row_bits(int L) {
+  return (kD / pages_g(L)) * pages_b(L) + (pages_tail(L) ? bits_for(ipow(L, pages_tail(L))) : 0);
+}
+// levels the decode reads in this layout: 2, 4 and 16 (their stream is the
+// word layout's), 8 (bit fields), and the levels whose groups split into at
+// most two parts that the f16 digit steps cover (3, 5, 6, 7, 10, 11, 13);
+// 9, 12, 14 and 15 would need a third part or a part beyond those steps
+__host__ __device__ constexpr bool pages_supported(int L) {
+  return L >= 2 && L <= 16 && L != 9 && L != 12 && L != 14 && L != 15;
+}
+
+// ---------------------------------------------------------------------------
 // Device status word
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void set_flag(uint32_t *status, uint32_t f) {

@@ -147,6 +147,58 @@ __host__ __device__ constexpr uint16_t f16_int_bits(int v) {
   return (uint16_t)((v < 0 ? 0x8000 : 0) | ((e + 15) << 10) | mant);
 }
 
+// ST f16 digit steps on the packed pair x = (1024 + Pa, 1024 + Pb): out[o0 + s]
+// = (digit s of Pa, digit s of Pb), least significant first
+template <int L, int ST, int NR>
+__device__ __forceinline__ void f16_digit_steps(uint32_t x, uint32_t (&out)[NR], int o0) {
+  constexpr uint32_t C0 = h2dup(f16_plan(L).c0), K0 = h2dup(f16_plan(L).k0);
+  constexpr uint32_t C1 = h2dup(f16_plan(L).c1), K1 = h2dup(f16_plan(L).k1);
+  constexpr uint32_t NEGL = h2dup(f16_int_bits(-L));
+  constexpr uint32_t R0 = h2dup(f16_int_bits(1536 * L - 1024)), R1 = h2dup(f16_int_bits(1536 * L - 1536));
+  constexpr uint32_t M1024 = h2dup(f16_int_bits(-1024)), M1536 = h2dup(f16_int_bits(-1536));
+  if constexpr (ST == 1) {
+    out[o0] = hadd2(x, M1024);
+  } else {
+    uint32_t t = hfma2(x, C0, K0);
+    out[o0] = hadd2(x, hfma2(t, NEGL, R0));
+#pragma unroll
+    for (int s = 1; s < ST - 1; ++s) {
+      const uint32_t t2 = hfma2(t, C1, K1);
+      out[o0 + s] = hadd2(t, hfma2(t2, NEGL, R1));
+      t = t2;
+    }
+    out[o0 + ST - 1] = hadd2(t, M1536);
+  }
+}
+
+// register pair J of a word (parts 2J, 2J+1) and the ones after it; `rest`
+// holds the word's digits from part 2J on
+template <int L, int J, int NR>
+__device__ __forceinline__ void extract_regs(uint32_t rest, uint32_t (&out)[NR], int o) {
+  if constexpr (J < plan_regs(L)) {
+    constexpr int ka = plan_part(L, 2 * J), kb = plan_part(L, 2 * J + 1);
+    uint32_t v = rest, next = 0;
+    if constexpr (J < plan_regs(L) - 1) {
+      constexpr uint32_t D = (uint32_t)ipow(L, ka + kb);
+      next = rest / D;
+      v = rest - next * D;
+    }
+    uint32_t x;
+    if constexpr (kb > 0) {
+      // (v mod L^ka) | (v div L^ka) << 16: the quotient by multiply-high is
+      // exact because v < L^(ka+kb) and L^ka * L^(ka+kb) < 2^32
+      constexpr uint32_t Da = (uint32_t)ipow(L, ka);
+      const uint32_t q = __umulhi(v, (uint32_t)((0x100000000ull + Da - 1) / Da));
+      x = (v + q * (65536u - Da)) | 0x64006400u;
+    } else {
+      x = v | 0x64006400u;
+    }
+    constexpr int st = ka > kb ? ka : kb;
+    f16_digit_steps<L, st>(x, out, o);
+    extract_regs<L, J + 1>(next, out, o + st);
+  }
+}
+
 // the S/2 digit-pair registers of word w, in slot order, into out[o0 ..]
 template <int L, int NR>
 __device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&out)[NR], int o0) {
@@ -160,51 +212,8 @@ __device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&out)[NR], in
 #pragma unroll
     for (int m = 1; m < 5; ++m) out[o0 + m] = ((w >> (3 * m)) & 7u) | ((w >> (3 * m - 1)) & 0x70000u);
   } else {
-    constexpr uint32_t C0 = h2dup(f16_plan(L).c0), K0 = h2dup(f16_plan(L).k0);
-    constexpr uint32_t C1 = h2dup(f16_plan(L).c1), K1 = h2dup(f16_plan(L).k1);
-    constexpr uint32_t NEGL = h2dup(f16_int_bits(-L));
-    constexpr uint32_t R0 = h2dup(f16_int_bits(1536 * L - 1024)), R1 = h2dup(f16_int_bits(1536 * L - 1536));
-    constexpr uint32_t M1024 = h2dup(f16_int_bits(-1024)), M1536 = h2dup(f16_int_bits(-1536));
     uint32_t rest = w;
-    int o = o0;
-#pragma unroll
-    for (int j = 0; j < plan_regs(L); ++j) {
-      const int ka = plan_part(L, 2 * j);
-      const int kb = plan_part(L, 2 * j + 1);
-      uint32_t v;
-      if (j < plan_regs(L) - 1) {
-        const uint32_t D = (uint32_t)ipow(L, ka + kb);
-        const uint32_t qq = rest / D;
-        v = rest - qq * D;
-        rest = qq;
-      } else {
-        v = rest;
-      }
-      uint32_t x;
-      if (kb > 0) {
-        // (v mod L^ka) | (v div L^ka) << 16: the quotient by multiply-high is
-        // exact because v < L^(ka+kb) and L^ka * L^(ka+kb) < 2^32
-        const uint32_t Da = (uint32_t)ipow(L, ka);
-        const uint32_t q = __umulhi(v, (uint32_t)((0x100000000ull + Da - 1) / Da));
-        x = (v + q * (65536u - Da)) | 0x64006400u;
-      } else {
-        x = v | 0x64006400u;
-      }
-      const int st = ka > kb ? ka : kb;
-      if (st == 1) {
-        out[o++] = hadd2(x, M1024);
-        continue;
-      }
-      uint32_t t = hfma2(x, C0, K0);
-      out[o++] = hadd2(x, hfma2(t, NEGL, R0));
-#pragma unroll
-      for (int s = 1; s < st - 1; ++s) {
-        const uint32_t t2 = hfma2(t, C1, K1);
-        out[o++] = hadd2(t, hfma2(t2, NEGL, R1));
-        t = t2;
-      }
-      out[o++] = hadd2(t, M1536);
-    }
+    extract_regs<L, 0>(rest, out, o0);
   }
 }
 
@@ -233,13 +242,120 @@ __device__ __forceinline__ int slot_dim(int c, int u) {
   return (u < G::WPG * G::SP && dg >= 0 && wi < G::W && d < kD) ? d : -1;
 }
 
+// ---- the pages' layout (SEMKV_LAYOUT_PAGES): rows are bit streams of groups
+// of g digits in b bits.  KIND 0: levels 2, 4, 16, whose stream is the word
+// layout's (read as words); KIND 1: a group splits into two f16 parts (ka, kb)
+// that share one register chain; KIND 2: a group is one part below 1024 and
+// two groups share a chain; KIND 3: level 8, digits are 3-bit fields.  A block
+// of groups (2, or 4 for KIND 2) fills whole k-blocks; the lane group c owns
+// blocks c*BPG .. c*BPG+BPG-1 of a row.
+template <int L>
+struct PGeo {
+  static constexpr int g = pages_g(L), b = pages_b(L), NGRP = pages_groups(L), R = pages_row_bits(L);
+  static constexpr int TD = kD - (NGRP - 1) * g;                       // digits of the last group
+  static constexpr int TB = bits_for(ipow(L, TD));                     // its bits
+  static constexpr int KIND = (L == 2 || L == 4 || L == 16) ? 0 : L == 8 ? 3 : (ipow(L, g) <= 1024 ? 2 : 1);
+  static constexpr int KA = (g + 1) / 2, KBP = g - KA;                 // KIND 1 parts
+  static constexpr int RPGR = KIND == 3 ? 3 : KA;                      // registers per group (KIND 1, 3)
+  static constexpr int GB = KIND == 2 ? 4 : 2;                         // groups per block
+  static constexpr int RB = KIND == 2 ? 2 * g : 2 * RPGR;              // registers per block
+  static constexpr int NBLK = (NGRP + GB - 1) / GB;
+  static constexpr int BPG = (NBLK + 3) / 4;                           // blocks per lane group
+  static constexpr int KB = BPG * RB / 2;                              // 16-slot k-blocks
+  static constexpr int TT = 32;
+  static constexpr int CW = ((TT * R + 31) / 32 + 16 + 3) / 4 * 4;     // staged stream words (+ copy slack)
+  static constexpr int TILE_BYTES = 2 * CW * 4 + 2 * TT * 4;
+  static constexpr float FAC = KIND == 3 ? 16777216.0f : 1.0f;
+  static_assert(KIND == 0 || RB % 2 == 0, "a block must fill whole k-block positions");
+  static_assert(!pages_supported(L) || KIND != 1 || (ipow(L, KA) <= 1024 && ipow(L, KA) * ipow(L, g) < (1ull << 32)),
+                "KIND 1 parts");
+};
+
+// b-bit field at stream bit `pos` of the staged buffer (pos >= 0, b <= 20)
+__device__ __forceinline__ uint32_t read_bits(const uint32_t *buf, int pos, int nbits) {
+  const int w = pos >> 5;
+  return __funnelshift_r(buf[w], buf[w + 1], pos & 31) & ((1u << nbits) - 1u);
+}
+
+// the RB digit-pair registers of block `blk` of the row whose stream starts at
+// buffer bit `rowbit`.  Groups past the row's last one read the bits after it:
+// every part stays below 2048, so those slots hold finite values, and they
+// carry q = 0 (K) or are never written out (V).
+template <int L>
+__device__ __forceinline__ void unpack_block(const uint32_t *buf, int rowbit, int blk,
+                                             uint32_t (&reg)[PGeo<L>::RB]) {
+  using P = PGeo<L>;
+  if constexpr (P::KIND == 1) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int gi = blk * 2 + q;
+      const uint32_t V = read_bits(buf, rowbit + gi * P::b, gi == P::NGRP - 1 ? P::TB : P::b);
+      constexpr uint32_t Da = (uint32_t)ipow(L, P::KA);
+      const uint32_t qq = __umulhi(V, (uint32_t)((0x100000000ull + Da - 1) / Da));
+      f16_digit_steps<L, P::KA>((V + qq * (65536u - Da)) | 0x64006400u, reg, q * P::KA);
+    }
+  } else if constexpr (P::KIND == 2) {
+#pragma unroll
+    for (int ch = 0; ch < 2; ++ch) {
+      const int g0 = blk * 4 + 2 * ch;
+      const uint32_t V0 = read_bits(buf, rowbit + g0 * P::b, g0 == P::NGRP - 1 ? P::TB : P::b);
+      const uint32_t V1 = read_bits(buf, rowbit + (g0 + 1) * P::b, g0 + 1 == P::NGRP - 1 ? P::TB : P::b);
+      f16_digit_steps<L, P::g>((V0 | (V1 << 16)) | 0x64006400u, reg, ch * P::g);
+    }
+  } else if constexpr (P::KIND == 3) {
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int gi = blk * 2 + q;
+      const uint32_t V = read_bits(buf, rowbit + gi * P::b, gi == P::NGRP - 1 ? P::TB : P::b);
+      reg[3 * q] = (V & 7u) | ((V << 13) & 0x70000u);              // digits 0, 1
+      reg[3 * q + 1] = ((V >> 6) & 7u) | ((V << 7) & 0x70000u);    // digits 2, 3
+      reg[3 * q + 2] = (V >> 12) & 7u;                              // digit 4
+    }
+  }
+}
+
+// head-dim index of slot u of lane group c in the pages' layout (or -1)
+template <int L>
+__device__ __forceinline__ int slot_dim_pages(int c, int u) {
+  using P = PGeo<L>;
+  const int blk = c * P::BPG + u / (2 * P::RB);
+  const int j = u % (2 * P::RB), m = j >> 1, h = j & 1;
+  int gi, dg, nd;
+  if constexpr (P::KIND == 2) {
+    gi = blk * 4 + 2 * (m / P::g) + h;
+    dg = m % P::g;
+    nd = gi == P::NGRP - 1 ? P::TD : P::g;
+  } else if constexpr (P::KIND == 3) {
+    gi = blk * 2 + m / 3;
+    dg = 2 * (m % 3) + h;
+    nd = gi == P::NGRP - 1 ? P::TD : P::g;
+  } else {
+    gi = blk * 2 + m / P::KA;
+    const int s = m % P::KA;
+    const int ka = (gi == P::NGRP - 1 && P::TD < P::KA) ? P::TD : P::KA;
+    const int kb = (gi == P::NGRP - 1 ? P::TD : P::g) - ka;
+    dg = h == 0 ? (s < ka ? s : -1) : (s < kb ? P::KA + s : -1);
+    nd = gi == P::NGRP - 1 ? P::TD : P::g;
+  }
+  const int d = gi * P::g + dg;
+  return (u < P::BPG * 2 * P::RB && gi < P::NGRP && dg >= 0 && dg < nd && d < kD) ? d : -1;
+}
+
+// slot map of either layout
+template <int L, bool GROUPS>
+__device__ __forceinline__ int slot_dim_any(int c, int u) {
+  if constexpr (GROUPS) return slot_dim_pages<L>(c, u);
+  else return slot_dim<L>(c, u);
+}
+
 // one pool class of a launch
 struct PoolArgs {
-  const uint32_t *kw, *vw;          // [B][Lyr][H][cap][W]
-  const float2 *km, *vm;            // [B][Lyr][H][cap]
+  const uint32_t *kw, *vw;          // [B][Lyr][H][slab_words] (words: [cap][W]; pages: bit stream)
+  const float2 *km, *vm;            // [B][Lyr][H][cap] (pages: __half2 per row)
   const int32_t *count;             // [B]
   int cap;
   int S, unit0;                     // splits per slab, first partial unit of this class
+  int64_t slab_words;               // code words of one (sequence, layer, head) slab
 };
 
 struct DecParams {
@@ -259,23 +375,31 @@ struct DecParams {
 };
 
 constexpr int kMergeBytes = DEC_WARPS * DEC_GMAX * kD * 4 + DEC_WARPS * DEC_GMAX * 3 * 4;
-template <int L>
-constexpr int kBarOff = (DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES > kMergeBytes)
-                            ? DEC_WARPS * DEC_NST * Geo<L>::TILE_BYTES : kMergeBytes;
-template <int L>
-constexpr int kQOff = kBarOff<L> + DEC_WARPS * DEC_NST * 8;
-static_assert(Geo<6>::TILE_BYTES % 16 == 0 && Geo<5>::TILE_BYTES % 16 == 0 && kMergeBytes % 16 == 0,
-              "tile buffers must keep 16-byte alignment for bulk copies");
 constexpr int kWaitLimit = 1 << 20;         // mbarrier polls before a copy is declared lost
-template <int L>
-constexpr int kQfragBytes = Geo<L>::KB * 32 * 8;   // q operand fragments, [kb][lane] x 2 words
+// shared-memory layout of a pool CTA: per-warp tile rings, their mbarriers, the
+// q fragments and the q rows
+template <int L, bool PAGES>
+struct Lay {
+  static constexpr bool GROUPS = PAGES && PGeo<L>::KIND != 0;          // read the pages' groups
+  static constexpr int TILE = GROUPS ? PGeo<L>::TILE_BYTES : (PAGES ? Geo<L>::TT * Geo<L>::W * 8 + Geo<L>::TT * 8
+                                                                     : Geo<L>::TILE_BYTES);
+  static constexpr int KB = GROUPS ? PGeo<L>::KB : Geo<L>::KB;
+  static constexpr int BAR = (DEC_WARPS * DEC_NST * TILE > kMergeBytes) ? DEC_WARPS * DEC_NST * TILE : kMergeBytes;
+  static constexpr int QOFF = BAR + DEC_WARPS * DEC_NST * 8;
+  static constexpr int QFRAG = KB * 32 * 8;                            // q operand fragments, [kb][lane] x 2 words
+  static_assert(TILE % 16 == 0 && kMergeBytes % 16 == 0, "tile buffers must keep 16-byte alignment for bulk copies");
+};
 
 // One CTA's share of one pool class: tiles [tb, te) of split `split` of slab `slab`.
-template <int L, bool ROT>
+template <int L, bool ROT, bool PAGES>
 __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa, int slab, int split,
                                           uint8_t *smem) {
   using Gm = Geo<L>;
-  constexpr int KB = Gm::KB, W = Gm::W;
+  using Ly = Lay<L, PAGES>;
+  using Pg = PGeo<L>;
+  constexpr bool GROUPS = Ly::GROUPS;            // the pages' groups (else 32-bit words)
+  constexpr int KB = Ly::KB, W = Gm::W;
+  constexpr float FAC = GROUPS ? Pg::FAC : Gm::FAC;
   constexpr float kappa = (L == 2) ? 0.5f : 1.0f;       // keeps p*scale inside f16 range
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
   const int h = slab % p.H, li = (slab / p.H) % p.nL, b = slab / (p.H * p.nL);
@@ -283,10 +407,10 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
   const int G = p.G;
 
   // ---- shared memory: per-warp tile rings, their mbarriers, then the q rows
-  uint8_t *ring = smem + warp * DEC_NST * Gm::TILE_BYTES;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarOff<L>) + warp * DEC_NST;
-  uint2 *qfrag = reinterpret_cast<uint2 *>(smem + kQOff<L>);                        // [KB][32]
-  float *qs = reinterpret_cast<float *>(smem + kQOff<L> + kQfragBytes<L>);            // [G][128]
+  uint8_t *ring = smem + warp * DEC_NST * Ly::TILE;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Ly::BAR) + warp * DEC_NST;
+  uint2 *qfrag = reinterpret_cast<uint2 *>(smem + Ly::QOFF);                          // [KB][32]
+  float *qs = reinterpret_cast<float *>(smem + Ly::QOFF + Ly::QFRAG);                // [G][128]
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < DEC_NST; ++s) mbar_init(&bars[s], 1);
@@ -330,7 +454,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
       float v[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int d = slot_dim<L>(c, 4 * kb + 2 * hh + e);
+        const int d = slot_dim_any<L, GROUPS>(c, 4 * kb + 2 * hh + e);
         v[e] = (rq < G && d >= 0) ? qs[rq * kD + d] : 0.0f;
         qsum += qlo ? 0.0f : v[e];
         if (qlo) v[e] = __fsub_rn(v[e], __half2float(__float2half_rn(v[e])));
@@ -344,7 +468,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
   qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
   const float c2k = ROT ? p.c2 * (1.0f / 128.0f) : p.c2;     // rotated: q' . k' / 128
   const float qsc = qsum * c2k;
-  const float kscale = c2k * Gm::FAC;                  // bit-field digits are c * 2^-24
+  const float kscale = c2k * FAC;                      // bit-field digits are c * 2^-24
   // This lane's two queries are the MMA columns 2c, 2c+1 of the logits.  With
   // G <= 4 columns 4..7 repeat heads 0..3 (or carry q''s low part when
   // rotated), so lane c >= 2 holds the same two heads as lane c-2 and the two
@@ -356,31 +480,46 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
   const float qs1 = __shfl_sync(0xffffffffu, qsc, 4 * (qc0 + 1));
 
   // ---- this CTA's tiles (32 tokens each)
-  constexpr int RPW = Gm::RPW, KPW = Gm::KPW, WPG = Gm::WPG, TT = Gm::TT;
+  constexpr int TT = Gm::TT;
+  constexpr int UPG = GROUPS ? Pg::BPG : Gm::WPG;     // units (words, or blocks of groups) per lane group
+  constexpr int RPU = GROUPS ? Pg::RB : Gm::RPW;      // f16x2 registers per unit
+  constexpr int KPU = RPU / 2;                        // k-blocks per unit
+  // staged tile: K codes, V codes, K meta, V meta (meta: 8 B a row, 4 B in the pages' layout)
+  constexpr int CWB = GROUPS ? Pg::CW * 4 : TT * W * 4;
+  constexpr int MB = PAGES ? 4 : 8;
   const int n = min(pa.count[b], pa.cap);
   const int ntile = (n + TT - 1) / TT;
   const int tb = (int)((int64_t)ntile * split / pa.S), te = (int)((int64_t)ntile * (split + 1) / pa.S);
-  const uint32_t *kw = pa.kw + pslab * pa.cap * W;
-  const uint32_t *vw = pa.vw + pslab * pa.cap * W;
-  const float2 *km = pa.km + pslab * pa.cap;
-  const float2 *vm = pa.vm + pslab * pa.cap;
+  const uint32_t *kw = pa.kw + pslab * pa.slab_words;
+  const uint32_t *vw = pa.vw + pslab * pa.slab_words;
+  const uint8_t *km = reinterpret_cast<const uint8_t *>(pa.km) + pslab * pa.cap * MB;
+  const uint8_t *vm = reinterpret_cast<const uint8_t *>(pa.vm) + pslab * pa.cap * MB;
 
   // one lane streams the warp's tiles: 4 bulk copies (K words, V words, K meta,
   // V meta) completing on the slot's mbarrier.  Capacities are multiples of
   // 16, so the last tile of a slab may hold 16 rows: the copies stop at the
   // capacity, and the rows of the buffer past it are masked like rows past n.
+  // In the pages' layout the tile's rows are stream bits [t0 R, (t0+nt) R): the
+  // copy takes the 16-byte aligned words around them, and the tile's first row
+  // starts at buffer bit (t0 R) mod 128.
   auto issue = [&](int tile, int slotix) {
     if (lane == 0 && tile < te) {
-      uint8_t *dst = ring + slotix * Gm::TILE_BYTES;
+      uint8_t *dst = ring + slotix * Ly::TILE;
       const int t0 = tile * TT;
       const int nt = min(TT, pa.cap - t0);
-      const uint32_t wb = (uint32_t)nt * W * 4;
+      int64_t w0 = (int64_t)t0 * W;
+      uint32_t wb = (uint32_t)nt * W * 4;
+      if constexpr (GROUPS) {
+        w0 = ((int64_t)t0 * Pg::R >> 5) & ~3ll;
+        const int64_t w1 = ((((int64_t)(t0 + nt) * Pg::R + 31) >> 5) + 3) & ~3ll;
+        wb = (uint32_t)(w1 - w0) * 4;
+      }
       fence_proxy_async_smem();
-      mbar_expect_tx(&bars[slotix], 2 * wb + (uint32_t)nt * 16);
-      bulk_g2s(dst, kw + (int64_t)t0 * W, wb, &bars[slotix]);
-      bulk_g2s(dst + TT * W * 4, vw + (int64_t)t0 * W, wb, &bars[slotix]);
-      bulk_g2s(dst + TT * W * 8, km + t0, (uint32_t)nt * 8, &bars[slotix]);
-      bulk_g2s(dst + TT * W * 8 + TT * 8, vm + t0, (uint32_t)nt * 8, &bars[slotix]);
+      mbar_expect_tx(&bars[slotix], 2 * wb + 2 * (uint32_t)nt * MB);
+      bulk_g2s(dst, kw + w0, wb, &bars[slotix]);
+      bulk_g2s(dst + CWB, vw + w0, wb, &bars[slotix]);
+      bulk_g2s(dst + 2 * CWB, km + (int64_t)t0 * MB, (uint32_t)nt * MB, &bars[slotix]);
+      bulk_g2s(dst + 2 * CWB + TT * MB, vm + (int64_t)t0 * MB, (uint32_t)nt * MB, &bars[slotix]);
     }
   };
 
@@ -413,28 +552,38 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
       break;
     }
     parity ^= 1u << slotix;
-    const uint8_t *tbuf = ring + slotix * Gm::TILE_BYTES;
+    const uint8_t *tbuf = ring + slotix * Ly::TILE;
     const uint32_t *sk = reinterpret_cast<const uint32_t *>(tbuf);
-    const uint32_t *sv = reinterpret_cast<const uint32_t *>(tbuf + TT * W * 4);
-    const float2 *skm = reinterpret_cast<const float2 *>(tbuf + TT * W * 8);
-    const float2 *svm = reinterpret_cast<const float2 *>(tbuf + TT * W * 8 + TT * 8);
+    const uint32_t *sv = reinterpret_cast<const uint32_t *>(tbuf + CWB);
+    const uint8_t *smk = tbuf + 2 * CWB, *smv = tbuf + 2 * CWB + TT * MB;
+    // (min, scale) of staged row tt
+    auto meta = [&](const uint8_t *base, int tt) -> float2 {
+      if constexpr (PAGES) return __half22float2(reinterpret_cast<const __half2 *>(base)[tt]);
+      else return reinterpret_cast<const float2 *>(base)[tt];
+    };
     const int t0 = tile * TT;
     const bool full = t0 + TT <= n;
+    const int rowbit0 = GROUPS ? (int)(((int64_t)t0 * Pg::R) & 127) : 0;
+    // the f16x2 digit registers of unit i of staged row `row`
+    auto unpack = [&](const uint32_t *buf, int row, int i, uint32_t (&regs)[RPU]) {
+      if constexpr (GROUPS) unpack_block<L>(buf, rowbit0 + row * Pg::R, c * UPG + i, regs);
+      else unpack_word<L>(buf[row * W + c * UPG + i], regs);
+    };
 
     // ---- logits S = C Q^T per 16-token block: tokens on the MMA rows (r, r+8),
     // query heads on the columns; each word goes to the tensor cores as soon
     // as it is unpacked
     float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-    for (int i = 0; i < WPG; ++i) {
+    for (int i = 0; i < UPG; ++i) {
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk) {
-        uint32_t ra[RPW], rb[RPW];
-        unpack_word<L>(sk[(blk * 16 + r) * W + c * WPG + i], ra);
-        unpack_word<L>(sk[(blk * 16 + 8 + r) * W + c * WPG + i], rb);
+        uint32_t ra[RPU], rb[RPU];
+        unpack(sk, blk * 16 + r, i, ra);
+        unpack(sk, blk * 16 + 8 + r, i, rb);
 #pragma unroll
-        for (int m = 0; m < KPW; ++m) {
-          const uint2 qb = qfrag[(i * KPW + m) * 32 + lane];
+        for (int m = 0; m < KPU; ++m) {
+          const uint2 qb = qfrag[(i * KPU + m) * 32 + lane];
           mma_16816(sacc[blk], ra[2 * m], rb[2 * m], ra[2 * m + 1], rb[2 * m + 1], qb.x, qb.y);
         }
       }
@@ -454,7 +603,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
         s4[i] = (pack_lo ? myblk : j) ? a1 : a0;
       }
       const int tt = (pack_lo ? myblk : j) * 16 + r;
-      const float2 m0 = skm[tt], m1 = skm[tt + 8];
+      const float2 m0 = meta(smk, tt), m1 = meta(smk, tt + 8);
       lg[j][0] = __fmaf_rn(s4[0], m0.y * kscale, m0.x * qs0);
       lg[j][1] = __fmaf_rn(s4[1], m0.y * kscale, m0.x * qs1);
       lg[j][2] = __fmaf_rn(s4[2], m1.y * kscale, m1.x * qs0);
@@ -509,7 +658,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
         const int tt = (pack_lo ? myblk : j) * 16 + 8 * g2 + r;
         const bool ok = full || t0 + tt < n;
         // rows past the count hold whatever the pool memory held: keep them out
-        const float2 vmm = ok ? svm[tt] : make_float2(0.0f, 0.0f);
+        const float2 vmm = ok ? meta(smv, tt) : make_float2(0.0f, 0.0f);
         float pw[2];
 #pragma unroll
         for (int e = 0; e < 2; ++e) {
@@ -550,15 +699,15 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
 
     // ---- values: O^T += C^T P' (codes transposed in registers), word by word
 #pragma unroll
-    for (int i = 0; i < WPG; ++i) {
+    for (int i = 0; i < UPG; ++i) {
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk) {
-        uint32_t ra[RPW], rb[RPW];
-        unpack_word<L>(sv[(blk * 16 + r) * W + c * WPG + i], ra);
-        unpack_word<L>(sv[(blk * 16 + 8 + r) * W + c * WPG + i], rb);
+        uint32_t ra[RPU], rb[RPU];
+        unpack(sv, blk * 16 + r, i, ra);
+        unpack(sv, blk * 16 + 8 + r, i, rb);
 #pragma unroll
-        for (int m = 0; m < KPW; ++m) {
-          const int kb = i * KPW + m;
+        for (int m = 0; m < KPU; ++m) {
+          const int kb = i * KPU + m;
           const uint32_t a0 = movmatrix_t(ra[2 * m]);
           const uint32_t a1 = movmatrix_t(ra[2 * m + 1]);
           const uint32_t a2 = movmatrix_t(rb[2 * m]);
@@ -614,7 +763,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
         wst[(warp * DEC_GMAX + qc0 + e) * 3 + 1] = l_run[e];
         wst[(warp * DEC_GMAX + qc0 + e) * 3 + 2] = mt_run[e];
       }
-  constexpr float unscale = Gm::FAC / kappa;
+  constexpr float unscale = FAC / kappa;
   if (owner)
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
@@ -622,7 +771,8 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
       for (int hh = 0; hh < 2; ++hh) {
         // slot r (hh=0) or 8+r (hh=1) of block kb belongs to lane group r/2, position (r%2) + 2hh
         // (both candidate slots are compile-time, so the slot table folds away)
-        const int dA = slot_dim<L>(r >> 1, 4 * kb + 2 * hh), dB = slot_dim<L>(r >> 1, 4 * kb + 2 * hh + 1);
+        const int dA = slot_dim_any<L, GROUPS>(r >> 1, 4 * kb + 2 * hh);
+        const int dB = slot_dim_any<L, GROUPS>(r >> 1, 4 * kb + 2 * hh + 1);
         const int d = (r & 1) ? dB : dA;
         if (d >= 0) {
           if (qc0 < G) wo[(warp * DEC_GMAX + qc0) * kD + d] = oacc[kb][2 * hh] * unscale;
@@ -659,7 +809,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
 // Both pool classes in one launch (LA: class 0 = high, LB: class 1 = low), so
 // that the CTAs of the two pools fill the same waves; a launch with one class
 // uses LA == LB.
-template <int LA, int LB, bool ROT>
+template <int LA, int LB, bool ROT, bool PAGES>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 4) decode_pool_kernel(const DecParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int n0 = p.slabs * p.pool[0].S;
@@ -667,10 +817,10 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 4) decode_pool_kernel(const De
   const int i = cls ? (int)blockIdx.x - n0 : (int)blockIdx.x;
   const int S = p.pool[cls].S;
   if constexpr (LA == LB) {
-    pool_body<LA, ROT>(p, p.pool[cls], i / S, i % S, smem);
+    pool_body<LA, ROT, PAGES>(p, p.pool[cls], i / S, i % S, smem);
   } else {
-    if (cls == 0) pool_body<LA, ROT>(p, p.pool[0], i / S, i % S, smem);
-    else pool_body<LB, ROT>(p, p.pool[1], i / S, i % S, smem);
+    if (cls == 0) pool_body<LA, ROT, PAGES>(p, p.pool[0], i / S, i % S, smem);
+    else pool_body<LB, ROT, PAGES>(p, p.pool[1], i / S, i % S, smem);
   }
 }
 
@@ -830,99 +980,133 @@ __global__ void decode_score_acc_kernel(const float *__restrict__ prob, int H_q,
 }
 
 // ---------------------------------------------------------------- host side
-template <int L>
+template <int L, bool PAGES>
 static int pool_smem_bytes(int G) {
-  return kQOff<L> + kQfragBytes<L> + G * kD * 4;
+  return Lay<L, PAGES>::QOFF + Lay<L, PAGES>::QFRAG + G * kD * 4;
 }
 
-template <int LA, int LB, bool ROT>
+// instances that exist: the pages' layout for its supported levels, unrotated
+template <int LA, int LB, bool ROT, bool PAGES>
+constexpr bool pools_instance() {
+  return !PAGES || (!ROT && pages_supported(LA) && pages_supported(LB));
+}
+
+template <int LA, int LB, bool ROT, bool PAGES>
 static cudaError_t launch_pools(const DecParams &p, int grid, cudaStream_t st) {
-  const int smem = pool_smem_bytes<LA>(p.G) > pool_smem_bytes<LB>(p.G) ? pool_smem_bytes<LA>(p.G)
-                                                                        : pool_smem_bytes<LB>(p.G);
-  const int smax = pool_smem_bytes<LA>(DEC_GMAX) > pool_smem_bytes<LB>(DEC_GMAX) ? pool_smem_bytes<LA>(DEC_GMAX)
-                                                                                : pool_smem_bytes<LB>(DEC_GMAX);
-  cudaError_t e = prepare_kernel(reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT>), smax);
-  if (e != cudaSuccess) return e;
-  if (grid > 0) decode_pool_kernel<LA, LB, ROT><<<grid, DEC_WARPS * 32, smem, st>>>(p);
-  return cudaGetLastError();
+  if constexpr (!pools_instance<LA, LB, ROT, PAGES>()) {
+    return cudaErrorInvalidValue;
+  } else {
+    const int sa = pool_smem_bytes<LA, PAGES>(p.G), sb = pool_smem_bytes<LB, PAGES>(p.G);
+    const int ma = pool_smem_bytes<LA, PAGES>(DEC_GMAX), mb = pool_smem_bytes<LB, PAGES>(DEC_GMAX);
+    const void *fn = reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT, PAGES>);
+    cudaError_t e = prepare_kernel(fn, ma > mb ? ma : mb);
+    if (e != cudaSuccess) return e;
+    if (grid > 0) decode_pool_kernel<LA, LB, ROT, PAGES><<<grid, DEC_WARPS * 32, sa > sb ? sa : sb, st>>>(p);
+    return cudaGetLastError();
+  }
 }
 
-// resident CTAs per SM of the kernel instance <LA, LB, ROT> (queried once per device)
-template <int LA, int LB, bool ROT>
+// resident CTAs per SM of the kernel instance <LA, LB, ROT, PAGES> (queried once per device)
+template <int LA, int LB, bool ROT, bool PAGES>
 static int pools_occupancy(int G) {
-  const int smem = pool_smem_bytes<LA>(G) > pool_smem_bytes<LB>(G) ? pool_smem_bytes<LA>(G) : pool_smem_bytes<LB>(G);
-  const int smax = pool_smem_bytes<LA>(DEC_GMAX) > pool_smem_bytes<LB>(DEC_GMAX) ? pool_smem_bytes<LA>(DEC_GMAX)
-                                                                                : pool_smem_bytes<LB>(DEC_GMAX);
-  const void *fn = reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT>);
-  int nb = 1;
-  if (prepare_kernel(fn, smax) != cudaSuccess || kernel_occupancy(fn, DEC_WARPS * 32, smem, &nb) != cudaSuccess)
+  if constexpr (!pools_instance<LA, LB, ROT, PAGES>()) {
     return 1;
-  return nb;
-}
-template <bool ROT>
-static int occupancy_one(int L, int G) {
-  switch (L) {
-    case 2: return pools_occupancy<2, 2, ROT>(G);
-    case 3: return pools_occupancy<3, 3, ROT>(G);
-    case 4: return pools_occupancy<4, 4, ROT>(G);
-    case 5: return pools_occupancy<5, 5, ROT>(G);
-    case 6: return pools_occupancy<6, 6, ROT>(G);
-    case 7: return pools_occupancy<7, 7, ROT>(G);
-    case 8: return pools_occupancy<8, 8, ROT>(G);
-    case 9: return pools_occupancy<9, 9, ROT>(G);
-    case 10: return pools_occupancy<10, 10, ROT>(G);
-    case 11: return pools_occupancy<11, 11, ROT>(G);
-    case 12: return pools_occupancy<12, 12, ROT>(G);
-    case 13: return pools_occupancy<13, 13, ROT>(G);
-    case 14: return pools_occupancy<14, 14, ROT>(G);
-    case 15: return pools_occupancy<15, 15, ROT>(G);
-    default: return pools_occupancy<16, 16, ROT>(G);
-  }
-}
-template <bool ROT>
-static int occupancy_merged(int Lh, int Ll, int G) {
-  if (Lh == Ll) return occupancy_one<ROT>(Lh, G);
-  if (Lh == 6 && Ll == 5) return pools_occupancy<6, 5, ROT>(G);
-  if (Lh == 5 && Ll == 4) return pools_occupancy<5, 4, ROT>(G);
-  if (Lh == 8 && Ll == 6) return pools_occupancy<8, 6, ROT>(G);
-  return pools_occupancy<16, 8, ROT>(G);
-}
-
-// one class per launch, any level
-template <bool ROT>
-static cudaError_t launch_one(int L, const DecParams &p, int grid, cudaStream_t st) {
-  switch (L) {
-    case 2: return launch_pools<2, 2, ROT>(p, grid, st);
-    case 3: return launch_pools<3, 3, ROT>(p, grid, st);
-    case 4: return launch_pools<4, 4, ROT>(p, grid, st);
-    case 5: return launch_pools<5, 5, ROT>(p, grid, st);
-    case 6: return launch_pools<6, 6, ROT>(p, grid, st);
-    case 7: return launch_pools<7, 7, ROT>(p, grid, st);
-    case 8: return launch_pools<8, 8, ROT>(p, grid, st);
-    case 9: return launch_pools<9, 9, ROT>(p, grid, st);
-    case 10: return launch_pools<10, 10, ROT>(p, grid, st);
-    case 11: return launch_pools<11, 11, ROT>(p, grid, st);
-    case 12: return launch_pools<12, 12, ROT>(p, grid, st);
-    case 13: return launch_pools<13, 13, ROT>(p, grid, st);
-    case 14: return launch_pools<14, 14, ROT>(p, grid, st);
-    case 15: return launch_pools<15, 15, ROT>(p, grid, st);
-    case 16: return launch_pools<16, 16, ROT>(p, grid, st);
-    default: return cudaErrorInvalidValue;
+  } else {
+    const int sa = pool_smem_bytes<LA, PAGES>(G), sb = pool_smem_bytes<LB, PAGES>(G);
+    const int ma = pool_smem_bytes<LA, PAGES>(DEC_GMAX), mb = pool_smem_bytes<LB, PAGES>(DEC_GMAX);
+    const void *fn = reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT, PAGES>);
+    int nb = 1;
+    if (prepare_kernel(fn, ma > mb ? ma : mb) != cudaSuccess ||
+        kernel_occupancy(fn, DEC_WARPS * 32, sa > sb ? sa : sb, &nb) != cudaSuccess)
+      return 1;
+    return nb;
   }
 }
 
+// F is called as f.template run<LA, LB>() for the instance of the levels
+template <typename F>
+static auto dispatch_one(int L, F &f) {
+  switch (L) {
+    case 2: return f.template run<2, 2>();
+    case 3: return f.template run<3, 3>();
+    case 4: return f.template run<4, 4>();
+    case 5: return f.template run<5, 5>();
+    case 6: return f.template run<6, 6>();
+    case 7: return f.template run<7, 7>();
+    case 8: return f.template run<8, 8>();
+    case 9: return f.template run<9, 9>();
+    case 10: return f.template run<10, 10>();
+    case 11: return f.template run<11, 11>();
+    case 12: return f.template run<12, 12>();
+    case 13: return f.template run<13, 13>();
+    case 14: return f.template run<14, 14>();
+    case 15: return f.template run<15, 15>();
+    default: return f.template run<16, 16>();
+  }
+}
 // both classes in one launch: every uniform pair, and the adjacent pairs the
 // pages use (6/5) or sweep (5/4, 8/6, 16/8); other pairs take two launches
 static bool has_merged(int Lh, int Ll) {
   return Lh == Ll || (Lh == 6 && Ll == 5) || (Lh == 5 && Ll == 4) || (Lh == 8 && Ll == 6) || (Lh == 16 && Ll == 8);
 }
-template <bool ROT>
-static cudaError_t launch_merged(int Lh, int Ll, const DecParams &p, int grid, cudaStream_t st) {
-  if (Lh == Ll) return launch_one<ROT>(Lh, p, grid, st);
-  if (Lh == 6 && Ll == 5) return launch_pools<6, 5, ROT>(p, grid, st);
-  if (Lh == 5 && Ll == 4) return launch_pools<5, 4, ROT>(p, grid, st);
-  if (Lh == 8 && Ll == 6) return launch_pools<8, 6, ROT>(p, grid, st);
-  return launch_pools<16, 8, ROT>(p, grid, st);
+template <typename F>
+static auto dispatch_merged(int Lh, int Ll, F &f) {
+  if (Lh == Ll) return dispatch_one(Lh, f);
+  if (Lh == 6 && Ll == 5) return f.template run<6, 5>();
+  if (Lh == 5 && Ll == 4) return f.template run<5, 4>();
+  if (Lh == 8 && Ll == 6) return f.template run<8, 6>();
+  return f.template run<16, 8>();
+}
+
+template <bool ROT, bool PAGES>
+struct LaunchF {
+  const DecParams &p;
+  int grid;
+  cudaStream_t st;
+  template <int LA, int LB>
+  cudaError_t run() { return launch_pools<LA, LB, ROT, PAGES>(p, grid, st); }
+};
+template <bool ROT, bool PAGES>
+struct OccF {
+  int G;
+  template <int LA, int LB>
+  int run() { return pools_occupancy<LA, LB, ROT, PAGES>(G); }
+};
+
+static cudaError_t launch_classes(bool merged, int Lh, int Ll, const semkv_cache &c, const DecParams &p, int grid,
+                                  cudaStream_t st) {
+  const int L = Lh;
+  (void)Ll;
+  if (c.layout == SEMKV_LAYOUT_PAGES) {
+    LaunchF<false, true> f{p, grid, st};
+    return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(L, f);
+  }
+  if (c.rotate) {
+    LaunchF<true, false> f{p, grid, st};
+    return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(L, f);
+  }
+  LaunchF<false, false> f{p, grid, st};
+  return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(L, f);
+}
+
+static int class_occupancy(bool merged, int Lh, int Ll, const semkv_cache &c) {
+  const int G = c.H_q / c.H;
+  if (c.layout == SEMKV_LAYOUT_PAGES) {
+    OccF<false, true> f{G};
+    return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(Lh, f);
+  }
+  if (c.rotate) {
+    OccF<true, false> f{G};
+    return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(Lh, f);
+  }
+  OccF<false, false> f{G};
+  return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(Lh, f);
+}
+
+// code words of one slab of a class
+static int64_t slab_words(const semkv_cache &c, int L, int cap) {
+  if (c.layout == SEMKV_LAYOUT_PAGES) return ((int64_t)cap * pages_row_bits(L) + 127) / 128 * 4;
+  return (int64_t)cap * words_per_row(L);
 }
 
 // Splits per slab of each class (the host knows only capacities).  CTAs of
@@ -934,13 +1118,12 @@ static cudaError_t launch_merged(int Lh, int Ll, const DecParams &p, int grid, c
 // gives 8 splits per pool, 4096 CTAs in 7 rounds of 592.
 static void pool_splits(const semkv_cache &c, int n_layers, int *Sh, int *Sl) {
   const bool merged = has_merged(c.L_high, c.L_low);
-  const int G = c.H_q / c.H;
   int occ;
   if (merged) {
-    occ = c.rotate ? occupancy_merged<true>(c.L_high, c.L_low, G) : occupancy_merged<false>(c.L_high, c.L_low, G);
+    occ = class_occupancy(true, c.L_high, c.L_low, c);
   } else {
-    const int oh = c.rotate ? occupancy_one<true>(c.L_high, G) : occupancy_one<false>(c.L_high, G);
-    const int ol = c.rotate ? occupancy_one<true>(c.L_low, G) : occupancy_one<false>(c.L_low, G);
+    const int oh = class_occupancy(false, c.L_high, c.L_high, c);
+    const int ol = class_occupancy(false, c.L_low, c.L_low, c);
     occ = oh < ol ? oh : ol;
   }
   const int64_t R = (int64_t)device_sm_count() * occ;
@@ -1003,15 +1186,16 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int sc
   p.rot = c.rotate;
   p.wait0 = first_wait_polls(kWaitLimit);
   const PoolArgs high = {c.k_high, c.v_high, reinterpret_cast<const float2 *>(c.k_high_meta),
-                         reinterpret_cast<const float2 *>(c.v_high_meta), c.n_high, c.cap_high, Sh, 0};
+                         reinterpret_cast<const float2 *>(c.v_high_meta), c.n_high, c.cap_high, Sh, 0,
+                         slab_words(c, c.L_high, c.cap_high)};
   const PoolArgs low = {c.k_low, c.v_low, reinterpret_cast<const float2 *>(c.k_low_meta),
-                        reinterpret_cast<const float2 *>(c.v_low_meta), c.n_low, c.cap_low, Sl, Sh};
+                        reinterpret_cast<const float2 *>(c.v_low_meta), c.n_low, c.cap_low, Sl, Sh,
+                        slab_words(c, c.L_low, c.cap_low)};
   cudaError_t e;
   if (has_merged(c.L_high, c.L_low)) {
     p.pool[0] = high;
     p.pool[1] = low;
-    e = c.rotate ? launch_merged<true>(c.L_high, c.L_low, p, slabs * (Sh + Sl), st)
-                 : launch_merged<false>(c.L_high, c.L_low, p, slabs * (Sh + Sl), st);
+    e = launch_classes(true, c.L_high, c.L_low, c, p, slabs * (Sh + Sl), st);
     if (e != cudaSuccess) return e;
   } else {
     for (int cls = 0; cls < 2; ++cls) {
@@ -1019,7 +1203,7 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int sc
       p.pool[1] = p.pool[0];
       p.pool[1].S = 0;
       const int L = cls ? c.L_low : c.L_high;
-      e = c.rotate ? launch_one<true>(L, p, slabs * p.pool[0].S, st) : launch_one<false>(L, p, slabs * p.pool[0].S, st);
+      e = launch_classes(false, L, L, c, p, slabs * p.pool[0].S, st);
       if (e != cudaSuccess) return e;
     }
   }

@@ -39,6 +39,7 @@ struct QuantLaunch {
   float *k_high_meta, *v_high_meta, *k_low_meta, *v_low_meta;
   int cap_high, cap_low, L_high, L_low;
   int rotate;                       // 1: Hadamard-rotate each row before quantizing
+  int layout;                       // SEMKV_LAYOUT_WORDS or SEMKV_LAYOUT_PAGES
   uint32_t *status;
 };
 cudaError_t launch_quantize(const QuantLaunch &q, cudaStream_t st);

@@ -39,6 +39,17 @@ def test_host_helpers_match_oracle(kv):
         assert kv.semkv_num_high(n, r) == O.num_high(n, r)
     assert kv.semkv_num_high(-1, 5) == -1 and kv.semkv_num_high(5, 1_000_001) == -1
     assert "sm_100a" in kv.semkv_version()
+    # storage sizes of both layouts (the pages' layout: rows back to back at bit granularity)
+    for L in range(2, 17):
+        assert kv.semkv_row_bits(kv.LAYOUT_WORDS, L) == 32 * O.words_per_row(L)
+        assert kv.semkv_pool_words(kv.LAYOUT_WORDS, L, 48) == 48 * O.words_per_row(L)
+        if L in (9, 12, 14, 15):
+            assert kv.semkv_row_bits(kv.LAYOUT_PAGES, L) == -1
+            continue
+        assert kv.semkv_row_bits(kv.LAYOUT_PAGES, L) == O.pages_row_bits(L)
+        assert kv.semkv_pool_words(kv.LAYOUT_PAGES, L, 48) * 4 >= (48 * O.pages_row_bits(L) + 7) // 8
+        assert kv.semkv_pool_words(kv.LAYOUT_PAGES, L, 48) % 4 == 0
+    assert kv.semkv_row_bits(2, 6) == -1 and kv.semkv_pool_words(kv.LAYOUT_PAGES, 6, -1) == -1
 
 
 def test_invalid_arguments_rejected_before_launch(kv):
@@ -51,17 +62,20 @@ def test_invalid_arguments_rejected_before_launch(kv):
     # a cache with D != 128, bad levels, unaligned pointers, bad capacities
     def cache(**kw):
         base = dict(B=1, n_layers=1, H=1, H_q=4, D=128, L_high=6, L_low=5, r_ppm=500_000, cap_high=16,
-                    cap_low=16, block=128, buf_len=0, rotate=0)
+                    cap_low=16, block=128, buf_len=0, rotate=0, layout=0)
         base.update(kw)
-        c = b.SemkvCache(*[base[k] for k in ("B", "n_layers", "H", "H_q", "D", "L_high", "L_low", "r_ppm",
-                                              "cap_high", "cap_low", "block", "buf_len", "rotate")])
-        for f, _ in b.SemkvCache._fields_[13:]:
+        names = ("B", "n_layers", "H", "H_q", "D", "L_high", "L_low", "r_ppm", "cap_high", "cap_low", "block",
+                 "buf_len", "rotate", "layout")
+        c = b.SemkvCache(*[base[k] for k in names])
+        for f, _ in b.SemkvCache._fields_[len(names):]:
             setattr(c, f, 0x10000)
         return c
     for kw, want in [(dict(D=64), UNSUP), (dict(L_high=17), UNSUP), (dict(L_low=1), UNSUP),
                      (dict(H_q=3, H=2), INVALID), (dict(H_q=36, H=4), UNSUP), (dict(r_ppm=-1), INVALID),
                      (dict(cap_high=17), INVALID), (dict(block=0), INVALID), (dict(buf_len=128), INVALID),
-                     (dict(rotate=2), INVALID), (dict(rotate=1, H_q=8, H=1), UNSUP)]:
+                     (dict(rotate=2), INVALID), (dict(rotate=1, H_q=8, H=1), UNSUP),
+                     (dict(layout=2), INVALID), (dict(layout=1, L_high=12), UNSUP),
+                     (dict(layout=1, L_low=9), UNSUP), (dict(layout=1, rotate=1), UNSUP)]:
         c = cache(**kw)
         assert b._lib_decode(ctypes.byref(c), 0, 1, ctypes.c_void_p(0x10000), ctypes.c_void_p(0x10000), 1.0,
                              ctypes.c_void_p(0x10000), 1 << 20, None, None) == want, kw
