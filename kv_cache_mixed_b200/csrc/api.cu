@@ -2,6 +2,7 @@
 // Everything here runs on the host; every GPU step is one of the kernels in
 // the other files of this directory.
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 #include <stdint.h>
 
 #include "../../include/semkv.h"
@@ -16,6 +17,14 @@ int first_wait_polls(int dflt) { return g_first_wait_polls < 0 ? dflt : g_first_
 }  // namespace semkv
 
 namespace {
+
+// An NVTX range around each call that enqueues GPU work, named after the call,
+// so a timeline tool shows which C-ABI call launched which kernels (a no-op
+// when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 inline bool al16(const void *p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -164,6 +173,7 @@ semkv_status semkv_score(int32_t kind, const uint16_t *k, int64_t k_batch_stride
                          const uint16_t *q_win, const int32_t *seq_len, int32_t B, int32_t T_max,
                          int32_t H, int32_t H_q, int32_t D, int32_t w, float *score, void *ws,
                          size_t ws_bytes, uint32_t *status, void *stream) {
+  NvtxRange nvtx_range("semkv_score");
   if (kind != SEMKV_SCORE_ATTN_MASS && kind != SEMKV_SCORE_KEY_L2) return SEMKV_ERR_INVALID_ARG;
   if (B <= 0 || T_max <= 0 || H <= 0) return SEMKV_ERR_INVALID_ARG;
   if (D != kD) return SEMKV_ERR_UNSUPPORTED;
@@ -189,6 +199,7 @@ semkv_status semkv_select(const float *score, int64_t score_batch_stride, const 
                           int32_t len_const, int32_t B, int32_t T_max, int32_t r_ppm, uint8_t *mask,
                           int64_t mask_batch_stride, void *ws, size_t ws_bytes, uint32_t *status,
                           void *stream) {
+  NvtxRange nvtx_range("semkv_select");
   (void)ws;
   (void)ws_bytes;
   if (B <= 0 || T_max <= 0 || r_ppm < 0 || r_ppm > 1000000) return SEMKV_ERR_INVALID_ARG;
@@ -208,6 +219,7 @@ size_t semkv_quantize_workspace_size(int32_t B, int32_t T_max) {
 semkv_status semkv_quantize(semkv_cache *c, const uint16_t *k, const uint16_t *v, int32_t T_max,
                             const int32_t *seq_len, const uint8_t *mask, void *ws, size_t ws_bytes,
                             uint32_t *status, void *stream) {
+  NvtxRange nvtx_range("semkv_quantize");
   semkv_status s = check_cache(c);
   if (s != SEMKV_OK) return s;
   if (T_max <= 0 || !al16(k) || !al16(v) || !al16(seq_len) || !al16(mask)) return SEMKV_ERR_INVALID_ARG;
@@ -224,6 +236,7 @@ size_t semkv_append_workspace_size(const semkv_cache *c) {
 semkv_status semkv_append_block(semkv_cache *c, const uint16_t *k_new, const uint16_t *v_new,
                                 const float *score_new, int32_t n, uint32_t flags, void *ws,
                                 size_t ws_bytes, uint32_t *status, void *stream) {
+  NvtxRange nvtx_range("semkv_append_block");
   semkv_status s = check_cache(c);
   if (s != SEMKV_OK) return s;
   if (n < 0 || (flags & ~SEMKV_FLUSH)) return SEMKV_ERR_INVALID_ARG;
@@ -268,12 +281,14 @@ static semkv_status decode_checked(const semkv_cache *c, int32_t layer0, int32_t
 semkv_status semkv_decode_attn(const semkv_cache *c, int32_t layer0, int32_t n_layers,
                                const uint16_t *q, uint16_t *out, float sm_scale, void *ws,
                                size_t ws_bytes, uint32_t *status, void *stream) {
+  NvtxRange nvtx_range("semkv_decode_attn");
   return decode_checked(c, layer0, n_layers, -1, q, out, sm_scale, ws, ws_bytes, status, stream);
 }
 
 semkv_status semkv_decode_attn_acc(const semkv_cache *c, int32_t layer0, int32_t n_layers,
                                    int32_t score_layer, const uint16_t *q, uint16_t *out, float sm_scale,
                                    void *ws, size_t ws_bytes, uint32_t *status, void *stream) {
+  NvtxRange nvtx_range("semkv_decode_attn_acc");
   if (c && (score_layer < layer0 || score_layer >= layer0 + n_layers)) return SEMKV_ERR_INVALID_ARG;
   if (c && c->buf_score == nullptr) return SEMKV_ERR_INVALID_ARG;
   return decode_checked(c, layer0, n_layers, score_layer, q, out, sm_scale, ws, ws_bytes, status, stream);

@@ -185,3 +185,39 @@ def test_decode_timeout_path_flags_and_recovers():
                 vals.append(np.concatenate(vh))
             ref[b, l] = O.decode_attn(qq[b, l], keys, vals)
     check_attention(to_np(out).astype(np.float64), ref)
+
+
+def test_decode_writes_only_its_outputs():
+    """Canaries around the decode outputs: a sentinel tail after `out` stays, the
+    pools and the query are read-only, and with score accumulation only the
+    FP16 block's first buf_len entries of buf_score change."""
+    kv = kv_mod()
+    wl = synth.scaled(synth.TINY, B=2, Lyr=3, H=2, H_q=8, T=300)
+    k, v = synth.kv(wl, 6, DEV)
+    score = synth.uniform_score(wl, 6, DEV)
+    seq_len = torch.tensor([300, 177], dtype=torch.int32, device=DEV)
+    mask = torch.zeros((2, 300), dtype=torch.uint8, device=DEV)
+    kv.semkv_select(score, seq_len, wl.r_ppm, mask)
+    cache = new_cache(2, 3, 2, 8, 6, 5, wl.r_ppm, 300, block=16)
+    kv.semkv_quantize(cache, k, v, seq_len, mask)
+    kn, vn, _ = synth.new_tokens(wl, 6, 0, DEV, n=5)
+    kv.semkv_append_block(cache, kn, vn, torch.rand((2, 5), device=DEV), 5)
+    cache.buf_score[:, 5:].fill_(-7.0)                       # entries past buf_len
+    pools_before = [t.clone() for t in (cache.k_high, cache.v_high, cache.k_low, cache.v_low,
+                                        cache.k_high_meta, cache.v_high_meta, cache.k_low_meta, cache.v_low_meta)]
+    q = synth.decode_query(wl, 6, DEV, n_layers=2)
+    q_before = q.clone()
+    n_out = q.numel()
+    out_full = torch.full((n_out + 4096,), 0x5A5A, dtype=torch.int16, device=DEV)
+    out = out_full[:n_out].view(torch.float16).view(q.shape)
+    kv.semkv_decode_attn_acc(cache, 1, 2, 2, q, out)          # layers 1..2, scores at layer 2
+    torch.cuda.synchronize()
+    assert cache.status_flags() == 0
+    assert torch.all(out_full[n_out:] == 0x5A5A)
+    assert torch.isfinite(out).all()
+    assert torch.equal(q, q_before)
+    for a, b in zip(pools_before, (cache.k_high, cache.v_high, cache.k_low, cache.v_low, cache.k_high_meta,
+                                   cache.v_high_meta, cache.k_low_meta, cache.v_low_meta)):
+        assert torch.equal(a, b)
+    bs = to_np(cache.buf_score)
+    assert np.all(bs[:, 5:] == -7.0)
