@@ -10,19 +10,30 @@
 // format of the MMA, so a digit is never converted after it is extracted.
 //
 // Digit extraction, levels that are not powers of two: a word is cut by
-// integer division into parts of k digits (L^k <= 1024), and two parts are
-// packed into one f16x2 register as the exact values 1024 + P (bit pattern
-// 0x6400 + P).  Then, on both halves at once, one f16 step
-//     t = fma(X, c, K)                 = 1536 + floor(P / L)   (exact; c, K below)
-//     digit = X + fma(t, -L, 1536 L - B) = P - L floor(P / L)   (exact)
-// peels the least significant digit off, and t is the next step's X (B is
-// X's bias: 1024 first, then 1536).  Every value stays an integer below 2048,
-// so each f16 operation is exact; (c, K) were chosen so that the rounding of
-// X c + K lands on 1536 + floor(P / L) for every part value, checked
-// exhaustively.  A step is three f16x2 instructions for two digits, all on
-// the FMA pipe.  Levels that are powers of two (2, 4, 8, 16) take their
-// digits straight out of the bit fields instead, as f16 subnormal patterns
-// c * 2^-24 (exact), with the 2^24 folded into the scales.
+// integer division into parts of k digits (L^k <= 1024), and two parts P are
+// packed into one f16x2 register.  Then, on both halves at once, one f16 step
+//     t = fma(X, c, K) = 1536 + floor(X' / L)     (X = 1024 + P first, then t)
+// gives the next floor of the part (exact: every value is an integer below
+// 2048, and (c, K) were chosen so that the rounding of X c + K lands on the
+// floor for every part value, checked exhaustively), and
+//     digit = X + fma(t, -L, 1536 L - B)     (B = X's bias, exact)
+// peels one digit off.
+//   Keys take the floors x_s = floor(P / L^s) themselves: the raw part P
+// (s = 0) costs nothing and a later floor is the low 9 bits of t, one logic
+// operation, so a step costs one f16x2 FMA and one logic operation for two
+// slots.  The digits d_s = x_s - L x_(s+1) are recovered by linearity on the
+// query side: slot s takes the coefficient q_s - L q_(s-1) (an f16 hi + lo
+// pair in the spare MMA columns), once per CTA.
+//   Values take the digits as normal f16 numbers.  The tensor cores add the
+// products into the accumulator by truncation, aligned to its exponent; with
+// subnormal value operands (v * 2^-24) the long value sums lost accuracy (the
+// worst full-size output error rose from 3.6e-4 to 8e-4 rel-L2), although a
+// single product of that size on its own comes out exact.
+//   Levels that are powers of two (2, 4, 8, 16) take their digits straight
+// out of the bit fields, placed 10 - log2 L bits up in an f16 subnormal
+// pattern (d * 2^(10 - log2 L - 24), exact), with the power of two folded
+// into the scales.  The pages' layout (groups in whole bits) feeds plain
+// digits through the digit chain.
 //
 // Work split: one pool class per launch (template on its L, and on whether
 // the rows are Hadamard-rotated); CTA = 4 warps on a contiguous range of
@@ -39,6 +50,8 @@
 // columns, with the digits and P' moved into that operand layout by
 // movmatrix.  With at most 4 query heads per KV head, columns 4..7 of the
 // value MMA carry the low f16 part of P', so one MMA takes both parts.
+#include <functional>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -111,6 +124,21 @@ __host__ __device__ constexpr int reg_digit(int L, int m, int h) {
   return -1;
 }
 
+// step s (floor(P / L^s)) of the part in half `h` of register m, or -1
+__host__ __device__ constexpr int reg_step(int L, int m, int h) {
+  if (is_pow2_level(L)) return -1;
+  int base = 0;
+  for (int j = 0; j < plan_regs(L); ++j) {
+    const int st = plan_steps(L, j);
+    if (m < base + st) {
+      const int pi = 2 * j + h, s = m - base;
+      return (pi < f16_plan(L).np && s < f16_plan(L).part[pi]) ? s : -1;
+    }
+    base += st;
+  }
+  return -1;
+}
+
 template <int L>
 struct Geo {
   static constexpr int N = digits_per_word(L);       // digits per word
@@ -123,8 +151,15 @@ struct Geo {
   static constexpr int KB = WPG * KPW;               // 16-slot k-blocks
   static constexpr int TT = 32;                      // tokens per tile (two 16-token MMA blocks)
   static constexpr int TILE_BYTES = TT * W * 4 * 2 + TT * 8 * 2;
-  // digits are f16 subnormal patterns c * 2^-24 on the bit-field path
-  static constexpr float FAC = is_pow2_level(L) ? 16777216.0f : 1.0f;
+  // bit-field digits (powers of two) sit SH bits up in an f16 subnormal
+  // pattern, d * 2^(SH-24), the highest place that keeps every digit below
+  // 2^10, so the value products stay as large as the bit fields allow (see
+  // the value digits above)
+  static constexpr int SH = is_pow2_level(L) ? 10 - bits_for(L) : 0;
+  // operand scales: keys take floors as subnormal patterns (x * 2^-24), values
+  // take normal f16 digits (levels that are not powers of two)
+  static constexpr float FAC_K = is_pow2_level(L) ? (float)(1 << (24 - SH)) : 16777216.0f;
+  static constexpr float FAC_V = is_pow2_level(L) ? (float)(1 << (24 - SH)) : 1.0f;
 };
 
 __device__ __forceinline__ uint32_t hfma2(uint32_t a, uint32_t b, uint32_t c) {
@@ -171,9 +206,33 @@ __device__ __forceinline__ void f16_digit_steps(uint32_t x, uint32_t (&out)[NR],
   }
 }
 
-// register pair J of a word (parts 2J, 2J+1) and the ones after it; `rest`
-// holds the word's digits from part 2J on
-template <int L, int J, int NR>
+// ST floor steps on the packed pair xb = (Pa, Pb) (two parts below 1024 as
+// raw 16-bit fields): out[o0 + s] = (floor(Pa / L^s), floor(Pb / L^s)) as f16
+// subnormal patterns, s = 0 .. ST-1.  The chain is the digit chain's first
+// half (X = 1024 + P, then t = 1536 + floor(P / L^s), exact); a floor below
+// 512 is then the low 9 bits of t's pattern 0x6600 + floor, one logic
+// operation.  Digits follow from the floors, d_s = x_s - L x_(s+1), which the
+// key side applies to q once instead of to every token.
+template <int L, int ST, int NR>
+__device__ __forceinline__ void f16_floor_steps(uint32_t xb, uint32_t (&out)[NR], int o0) {
+  constexpr uint32_t C0 = h2dup(f16_plan(L).c0), K0 = h2dup(f16_plan(L).k0);
+  constexpr uint32_t C1 = h2dup(f16_plan(L).c1), K1 = h2dup(f16_plan(L).k1);
+  out[o0] = xb;
+  if constexpr (ST > 1) {
+    uint32_t t = hfma2(xb | 0x64006400u, C0, K0);
+    out[o0 + 1] = t & 0x01ff01ffu;
+#pragma unroll
+    for (int s = 2; s < ST; ++s) {
+      t = hfma2(t, C1, K1);
+      out[o0 + s] = t & 0x01ff01ffu;
+    }
+  }
+}
+
+// register pair J of a word (parts 2J, 2J+1) and the ones after it: the
+// parts' floors (keys) or their digits (values); `rest` holds the
+// word's digits from part 2J on
+template <int L, int J, bool KEYS, int NR>
 __device__ __forceinline__ void extract_regs(uint32_t rest, uint32_t (&out)[NR], int o) {
   if constexpr (J < plan_regs(L)) {
     constexpr int ka = plan_part(L, 2 * J), kb = plan_part(L, 2 * J + 1);
@@ -183,37 +242,42 @@ __device__ __forceinline__ void extract_regs(uint32_t rest, uint32_t (&out)[NR],
       next = rest / D;
       v = rest - next * D;
     }
-    uint32_t x;
+    uint32_t xb;
     if constexpr (kb > 0) {
       // (v mod L^ka) | (v div L^ka) << 16: the quotient by multiply-high is
       // exact because v < L^(ka+kb) and L^ka * L^(ka+kb) < 2^32
       constexpr uint32_t Da = (uint32_t)ipow(L, ka);
       const uint32_t q = __umulhi(v, (uint32_t)((0x100000000ull + Da - 1) / Da));
-      x = (v + q * (65536u - Da)) | 0x64006400u;
+      xb = v + q * (65536u - Da);
     } else {
-      x = v | 0x64006400u;
+      xb = v;
     }
     constexpr int st = ka > kb ? ka : kb;
-    f16_digit_steps<L, st>(x, out, o);
-    extract_regs<L, J + 1>(next, out, o + st);
+    if constexpr (KEYS) f16_floor_steps<L, st>(xb, out, o);
+    else f16_digit_steps<L, st>(xb | 0x64006400u, out, o);
+    extract_regs<L, J + 1, KEYS>(next, out, o + st);
   }
 }
 
-// the S/2 digit-pair registers of word w, in slot order, into out[o0 ..]
-template <int L, int NR>
+// the S/2 operand registers of word w, in slot order, into out[o0 ..]: bit
+// fields as d << SH subnormal patterns (powers of two), else the parts' floors
+// (keys) or digits (values)
+template <int L, bool KEYS, int NR>
 __device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&out)[NR], int o0) {
+  constexpr int SH = Geo<L>::SH;
+  // bits [at, at + b) of w moved to bit `to`
+  auto field = [&](int at, int to) -> uint32_t { return at >= to ? (w >> (at - to)) : (w << (to - at)); };
   if constexpr (L == 2 || L == 4 || L == 16) {
     constexpr int b = L == 2 ? 1 : (L == 4 ? 2 : 4);
-    constexpr uint32_t msk = (uint32_t)(L - 1) * 0x00010001u;
+    constexpr uint32_t msk = ((uint32_t)(L - 1) * 0x00010001u) << SH;
 #pragma unroll
-    for (int m = 0; m < 16 / b; ++m) out[o0 + m] = (w >> (b * m)) & msk;   // digits m, m + 16/b
+    for (int m = 0; m < 16 / b; ++m) out[o0 + m] = field(b * m, SH) & msk;          // digits m, m + 16/b
   } else if constexpr (L == 8) {
-    out[o0] = (w & 7u) | ((w << 1) & 0x70000u);                              // digits 0, 5
 #pragma unroll
-    for (int m = 1; m < 5; ++m) out[o0 + m] = ((w >> (3 * m)) & 7u) | ((w >> (3 * m - 1)) & 0x70000u);
+    for (int m = 0; m < 5; ++m)                                                       // digits m, m + 5
+      out[o0 + m] = (field(3 * m, SH) & (7u << SH)) | (field(3 * m + 15, 16 + SH) & (7u << (16 + SH)));
   } else {
-    uint32_t rest = w;
-    extract_regs<L, 0>(rest, out, o0);
+    extract_regs<L, 0, KEYS>(w, out, o0);
   }
 }
 
@@ -224,9 +288,9 @@ __device__ __forceinline__ void extract_word(uint32_t w, uint32_t (&out)[NR], in
 // tensor cores as soon as it is unpacked.  Words past W of the row read the
 // next bytes of the tile buffer: every part of any 32-bit value stays a
 // finite f16, and those slots carry q = 0 (K) or are never written out (V).
-template <int L>
+template <int L, bool KEYS>
 __device__ __forceinline__ void unpack_word(uint32_t w, uint32_t (&reg)[Geo<L>::RPW]) {
-  extract_word<L, Geo<L>::RPW>(w, reg, 0);
+  extract_word<L, KEYS, Geo<L>::RPW>(w, reg, 0);
 #pragma unroll
   for (int u = Geo<L>::S / 2; u < Geo<L>::RPW; ++u) reg[u] = 0u;
 }
@@ -240,6 +304,15 @@ __device__ __forceinline__ int slot_dim(int c, int u) {
   const int dg = j < G::S ? reg_digit(L, j >> 1, j & 1) : -1;
   const int d = wi * G::N + dg;
   return (u < G::WPG * G::SP && dg >= 0 && wi < G::W && d < kD) ? d : -1;
+}
+
+// floor step of slot u of lane group c (levels that are not powers of two);
+// slot u holds floor(P / L^s) of the part whose digit s is slot_dim(c, u)
+template <int L>
+__device__ __forceinline__ int slot_step(int c, int u) {
+  using G = Geo<L>;
+  const int j = u % G::SP;
+  return j < G::S ? reg_step(L, j >> 1, j & 1) : -1;
 }
 
 // ---- the pages' layout (SEMKV_LAYOUT_PAGES): rows are bit streams of groups
@@ -378,28 +451,34 @@ constexpr int kMergeBytes = DEC_WARPS * DEC_GMAX * kD * 4 + DEC_WARPS * DEC_GMAX
 constexpr int kWaitLimit = 1 << 20;         // mbarrier polls before a copy is declared lost
 // shared-memory layout of a pool CTA: per-warp tile rings, their mbarriers, the
 // q fragments and the q rows
-template <int L, bool PAGES>
+template <int L, bool PAGES, bool WIDE>
 struct Lay {
   static constexpr bool GROUPS = PAGES && PGeo<L>::KIND != 0;          // read the pages' groups
   static constexpr int TILE = GROUPS ? PGeo<L>::TILE_BYTES : (PAGES ? Geo<L>::TT * Geo<L>::W * 8 + Geo<L>::TT * 8
                                                                      : Geo<L>::TILE_BYTES);
   static constexpr int KB = GROUPS ? PGeo<L>::KB : Geo<L>::KB;
+  static constexpr bool FLOORS = !GROUPS && !is_pow2_level(L);        // key slots hold floors, not digits
   static constexpr int BAR = (DEC_WARPS * DEC_NST * TILE > kMergeBytes) ? DEC_WARPS * DEC_NST * TILE : kMergeBytes;
   static constexpr int QOFF = BAR + DEC_WARPS * DEC_NST * 8;
-  static constexpr int QFRAG = KB * 32 * 8;                            // q operand fragments, [kb][lane] x 2 words
+  // q operand fragments, [kb][lane] x 2 words; with floors and G > 4 a second
+  // set holds the low f16 parts (they cannot ride in columns 4..7)
+  static constexpr int QFRAG = KB * 32 * 8 * (FLOORS && WIDE ? 2 : 1);
   static_assert(TILE % 16 == 0 && kMergeBytes % 16 == 0, "tile buffers must keep 16-byte alignment for bulk copies");
 };
 
-// One CTA's share of one pool class: tiles [tb, te) of split `split` of slab `slab`.
-template <int L, bool ROT, bool PAGES>
+// One CTA's share of one pool class: tiles [tb, te) of split `split` of slab
+// `slab`.  WIDE: more than 4 query heads per KV head (G > 4).
+template <int L, bool ROT, bool PAGES, bool WIDE>
 __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa, int slab, int split,
                                           uint8_t *smem) {
   using Gm = Geo<L>;
-  using Ly = Lay<L, PAGES>;
+  using Ly = Lay<L, PAGES, WIDE>;
   using Pg = PGeo<L>;
   constexpr bool GROUPS = Ly::GROUPS;            // the pages' groups (else 32-bit words)
+  constexpr bool FLOORS = Ly::FLOORS;            // key slots hold floor(P / L^s), not digits
   constexpr int KB = Ly::KB, W = Gm::W;
-  constexpr float FAC = GROUPS ? Pg::FAC : Gm::FAC;
+  constexpr float FAC_K = GROUPS ? Pg::FAC : Gm::FAC_K;          // operand scales, keys and values
+  constexpr float FAC_V = GROUPS ? Pg::FAC : Gm::FAC_V;
   constexpr float kappa = (L == 2) ? 0.5f : 1.0f;       // keeps p*scale inside f16 range
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, r = lane >> 2, c = lane & 3;
   const int h = slab % p.H, li = (slab / p.H) % p.nL, b = slab / (p.H * p.nL);
@@ -438,43 +517,61 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
 
   // ---- q fragments in slot order (kept in shared memory, one copy per CTA:
   // every warp uses the same fragments), and sum(q) * c2 for this lane's query r
-  // With rotated rows q' is not an f16 value: columns 0..3 carry its f16
-  // high part and columns 4..7 (G <= 4) its low part, q' - hi, so one MMA
-  // gives the logit to about 2^-22 relative.
-  // Without rotation and with G <= 4, columns 4..7 repeat the query heads of
-  // columns 0..3, so every lane of a row gets the logits of its head pair.
+  // A slot's coefficient is q_d for a digit slot.  For a floor slot x_s of a
+  // part it is q_d - L q_(d-1) for s >= 1 (d-1: the part's previous digit)
+  // and q_d for s = 0, since sum_s q_s d_s = q_0 x_0 + sum_(s>=1) (q_s - L
+  // q_(s-1)) x_s over a part's floors x_s = floor(P / L^s).
+  // A coefficient that is not an f16 value (rotated rows, floor slots) goes as
+  // an f16 pair hi + lo, to about 2^-22 relative: with G <= 4 columns 0..3
+  // carry hi and columns 4..7 lo, so one MMA takes both; with G > 4 the lo
+  // parts get MMAs of their own (second fragment set).
+  // Otherwise, with G <= 4, columns 4..7 repeat the query heads of columns
+  // 0..3, so every lane of a row gets the logits of its head pair.
   float qsum = 0.0f;
-  const bool qlo = ROT && r >= 4;
-  const int rq = (ROT || G <= 4) ? (r & 3) : r;
+  constexpr bool lo_cols = (ROT || FLOORS) && !WIDE;
+  constexpr bool lo_pass = FLOORS && WIDE;
+  const bool qlo = lo_cols && r >= 4;
+  const int rq = WIDE ? r : (r & 3);
 #pragma unroll
   for (int kb = 0; kb < KB; ++kb) {
-    uint32_t qv[2];
+    uint32_t qv[2], ql[2];
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
-      float v[2];
+      float v[2], vl[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int d = slot_dim_any<L, GROUPS>(c, 4 * kb + 2 * hh + e);
-        v[e] = (rq < G && d >= 0) ? qs[rq * kD + d] : 0.0f;
-        qsum += qlo ? 0.0f : v[e];
-        if (qlo) v[e] = __fsub_rn(v[e], __half2float(__float2half_rn(v[e])));
+        const int u = 4 * kb + 2 * hh + e;
+        const int d = slot_dim_any<L, GROUPS>(c, u);
+        const bool ok = rq < G && d >= 0;
+        const float qd = ok ? qs[rq * kD + d] : 0.0f;
+        float cf = qd;
+        if constexpr (FLOORS) {
+          if (ok && slot_step<L>(c, u) > 0) cf = __fmaf_rn(-(float)L, qs[rq * kD + d - 1], qd);
+        }
+        qsum += qlo ? 0.0f : qd;
+        vl[e] = __fsub_rn(cf, __half2float(__float2half_rn(cf)));
+        v[e] = qlo ? vl[e] : cf;
       }
       qv[hh] = pack_half2(v[0], v[1]);
+      ql[hh] = pack_half2(vl[0], vl[1]);
     }
-    if (warp == 0) qfrag[kb * 32 + lane] = make_uint2(qv[0], qv[1]);
+    if (warp == 0) {
+      qfrag[kb * 32 + lane] = make_uint2(qv[0], qv[1]);
+      if constexpr (lo_pass) qfrag[(KB + kb) * 32 + lane] = make_uint2(ql[0], ql[1]);
+    }
   }
   __syncthreads();
   qsum += __shfl_xor_sync(0xffffffffu, qsum, 1);
   qsum += __shfl_xor_sync(0xffffffffu, qsum, 2);
   const float c2k = ROT ? p.c2 * (1.0f / 128.0f) : p.c2;     // rotated: q' . k' / 128
   const float qsc = qsum * c2k;
-  const float kscale = c2k * FAC;                      // bit-field digits are c * 2^-24
+  const float kscale = c2k * FAC_K;                    // key operands are v / FAC_K
   // This lane's two queries are the MMA columns 2c, 2c+1 of the logits.  With
   // G <= 4 columns 4..7 repeat heads 0..3 (or carry q''s low part when
   // rotated), so lane c >= 2 holds the same two heads as lane c-2 and the two
   // lanes split each tile's blocks; the value MMA's columns 4..7 carry the low
   // f16 part of P', so one MMA per k-block takes both parts.
-  const bool pack_lo = G <= 4;
+  constexpr bool pack_lo = !WIDE;
   const int qc0 = pack_lo ? ((2 * c) & 3) : 2 * c;
   const float qs0 = __shfl_sync(0xffffffffu, qsc, 4 * qc0);        // sum(q)*c2 lives in quad r
   const float qs1 = __shfl_sync(0xffffffffu, qsc, 4 * (qc0 + 1));
@@ -564,11 +661,17 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
     const int t0 = tile * TT;
     const bool full = t0 + TT <= n;
     const int rowbit0 = GROUPS ? (int)(((int64_t)t0 * Pg::R) & 127) : 0;
-    // the f16x2 digit registers of unit i of staged row `row`
-    auto unpack = [&](const uint32_t *buf, int row, int i, uint32_t (&regs)[RPU]) {
-      if constexpr (GROUPS) unpack_block<L>(buf, rowbit0 + row * Pg::R, c * UPG + i, regs);
-      else unpack_word<L>(buf[row * W + c * UPG + i], regs);
+    // the f16x2 operand registers of unit i of staged row `row` (keys: the
+    // parts' floors; values: digits)
+    auto unpack = [&](bool keys, const uint32_t *buf, int row, int i, uint32_t (&regs)[RPU]) {
+      if constexpr (GROUPS) {
+        unpack_block<L>(buf, rowbit0 + row * Pg::R, c * UPG + i, regs);
+      } else {
+        if (keys) unpack_word<L, true>(buf[row * W + c * UPG + i], regs);
+        else unpack_word<L, false>(buf[row * W + c * UPG + i], regs);
+      }
     };
+    constexpr bool KEYS = true, VALUES = false;
 
     // ---- logits S = C Q^T per 16-token block: tokens on the MMA rows (r, r+8),
     // query heads on the columns; each word goes to the tensor cores as soon
@@ -579,12 +682,16 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk) {
         uint32_t ra[RPU], rb[RPU];
-        unpack(sk, blk * 16 + r, i, ra);
-        unpack(sk, blk * 16 + 8 + r, i, rb);
+        unpack(KEYS, sk, blk * 16 + r, i, ra);
+        unpack(KEYS, sk, blk * 16 + 8 + r, i, rb);
 #pragma unroll
         for (int m = 0; m < KPU; ++m) {
           const uint2 qb = qfrag[(i * KPU + m) * 32 + lane];
           mma_16816(sacc[blk], ra[2 * m], rb[2 * m], ra[2 * m + 1], rb[2 * m + 1], qb.x, qb.y);
+          if constexpr (lo_pass) {
+            const uint2 qc = qfrag[(KB + i * KPU + m) * 32 + lane];
+            mma_16816(sacc[blk], ra[2 * m], rb[2 * m], ra[2 * m + 1], rb[2 * m + 1], qc.x, qc.y);
+          }
         }
       }
     }
@@ -596,7 +703,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         float a0 = sacc[0][i], a1 = sacc[1][i];
-        if (ROT) {                                    // high + low part of q'
+        if constexpr (lo_cols) {                      // high + low part of the coefficients
           a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
           a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
         }
@@ -703,8 +810,8 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
 #pragma unroll
       for (int blk = 0; blk < 2; ++blk) {
         uint32_t ra[RPU], rb[RPU];
-        unpack(sv, blk * 16 + r, i, ra);
-        unpack(sv, blk * 16 + 8 + r, i, rb);
+        unpack(VALUES, sv, blk * 16 + r, i, ra);
+        unpack(VALUES, sv, blk * 16 + 8 + r, i, rb);
 #pragma unroll
         for (int m = 0; m < KPU; ++m) {
           const int kb = i * KPU + m;
@@ -713,7 +820,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
           const uint32_t a2 = movmatrix_t(rb[2 * m]);
           const uint32_t a3 = movmatrix_t(rb[2 * m + 1]);
           mma_16816(oacc[kb], a0, a1, a2, a3, bh[blk][0], bh[blk][1]);
-          if (!pack_lo) mma_16816(oacc[kb], a0, a1, a2, a3, bl[blk][0], bl[blk][1]);
+          if constexpr (!pack_lo) mma_16816(oacc[kb], a0, a1, a2, a3, bl[blk][0], bl[blk][1]);
         }
       }
     }
@@ -763,7 +870,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
         wst[(warp * DEC_GMAX + qc0 + e) * 3 + 1] = l_run[e];
         wst[(warp * DEC_GMAX + qc0 + e) * 3 + 2] = mt_run[e];
       }
-  constexpr float unscale = FAC / kappa;
+  constexpr float unscale = FAC_V / kappa;
   if (owner)
 #pragma unroll
     for (int kb = 0; kb < KB; ++kb) {
@@ -809,7 +916,7 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
 // Both pool classes in one launch (LA: class 0 = high, LB: class 1 = low), so
 // that the CTAs of the two pools fill the same waves; a launch with one class
 // uses LA == LB.
-template <int LA, int LB, bool ROT, bool PAGES>
+template <int LA, int LB, bool ROT, bool PAGES, bool WIDE>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 4) decode_pool_kernel(const DecParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int n0 = p.slabs * p.pool[0].S;
@@ -817,10 +924,10 @@ __global__ void __launch_bounds__(DEC_WARPS * 32, 4) decode_pool_kernel(const De
   const int i = cls ? (int)blockIdx.x - n0 : (int)blockIdx.x;
   const int S = p.pool[cls].S;
   if constexpr (LA == LB) {
-    pool_body<LA, ROT, PAGES>(p, p.pool[cls], i / S, i % S, smem);
+    pool_body<LA, ROT, PAGES, WIDE>(p, p.pool[cls], i / S, i % S, smem);
   } else {
-    if (cls == 0) pool_body<LA, ROT, PAGES>(p, p.pool[0], i / S, i % S, smem);
-    else pool_body<LB, ROT, PAGES>(p, p.pool[1], i / S, i % S, smem);
+    if (cls == 0) pool_body<LA, ROT, PAGES, WIDE>(p, p.pool[0], i / S, i % S, smem);
+    else pool_body<LB, ROT, PAGES, WIDE>(p, p.pool[1], i / S, i % S, smem);
   }
 }
 
@@ -980,41 +1087,42 @@ __global__ void decode_score_acc_kernel(const float *__restrict__ prob, int H_q,
 }
 
 // ---------------------------------------------------------------- host side
-template <int L, bool PAGES>
+template <int L, bool PAGES, bool WIDE>
 static int pool_smem_bytes(int G) {
-  return Lay<L, PAGES>::QOFF + Lay<L, PAGES>::QFRAG + G * kD * 4;
+  return Lay<L, PAGES, WIDE>::QOFF + Lay<L, PAGES, WIDE>::QFRAG + G * kD * 4;
 }
 
-// instances that exist: the pages' layout for its supported levels, unrotated
-template <int LA, int LB, bool ROT, bool PAGES>
+// instances that exist: the pages' layout for its supported levels, unrotated;
+// rotation only with G <= 4
+template <int LA, int LB, bool ROT, bool PAGES, bool WIDE>
 constexpr bool pools_instance() {
-  return !PAGES || (!ROT && pages_supported(LA) && pages_supported(LB));
+  return (!PAGES || (!ROT && pages_supported(LA) && pages_supported(LB))) && !(ROT && WIDE);
 }
 
-template <int LA, int LB, bool ROT, bool PAGES>
+template <int LA, int LB, bool ROT, bool PAGES, bool WIDE>
 static cudaError_t launch_pools(const DecParams &p, int grid, cudaStream_t st) {
-  if constexpr (!pools_instance<LA, LB, ROT, PAGES>()) {
+  if constexpr (!pools_instance<LA, LB, ROT, PAGES, WIDE>()) {
     return cudaErrorInvalidValue;
   } else {
-    const int sa = pool_smem_bytes<LA, PAGES>(p.G), sb = pool_smem_bytes<LB, PAGES>(p.G);
-    const int ma = pool_smem_bytes<LA, PAGES>(DEC_GMAX), mb = pool_smem_bytes<LB, PAGES>(DEC_GMAX);
-    const void *fn = reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT, PAGES>);
+    const int sa = pool_smem_bytes<LA, PAGES, WIDE>(p.G), sb = pool_smem_bytes<LB, PAGES, WIDE>(p.G);
+    const int ma = pool_smem_bytes<LA, PAGES, WIDE>(DEC_GMAX), mb = pool_smem_bytes<LB, PAGES, WIDE>(DEC_GMAX);
+    const void *fn = reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT, PAGES, WIDE>);
     cudaError_t e = prepare_kernel(fn, ma > mb ? ma : mb);
     if (e != cudaSuccess) return e;
-    if (grid > 0) decode_pool_kernel<LA, LB, ROT, PAGES><<<grid, DEC_WARPS * 32, sa > sb ? sa : sb, st>>>(p);
+    if (grid > 0) decode_pool_kernel<LA, LB, ROT, PAGES, WIDE><<<grid, DEC_WARPS * 32, sa > sb ? sa : sb, st>>>(p);
     return cudaGetLastError();
   }
 }
 
-// resident CTAs per SM of the kernel instance <LA, LB, ROT, PAGES> (queried once per device)
-template <int LA, int LB, bool ROT, bool PAGES>
+// resident CTAs per SM of the kernel instance <LA, LB, ROT, PAGES, WIDE> (queried once per device)
+template <int LA, int LB, bool ROT, bool PAGES, bool WIDE>
 static int pools_occupancy(int G) {
-  if constexpr (!pools_instance<LA, LB, ROT, PAGES>()) {
+  if constexpr (!pools_instance<LA, LB, ROT, PAGES, WIDE>()) {
     return 1;
   } else {
-    const int sa = pool_smem_bytes<LA, PAGES>(G), sb = pool_smem_bytes<LB, PAGES>(G);
-    const int ma = pool_smem_bytes<LA, PAGES>(DEC_GMAX), mb = pool_smem_bytes<LB, PAGES>(DEC_GMAX);
-    const void *fn = reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT, PAGES>);
+    const int sa = pool_smem_bytes<LA, PAGES, WIDE>(G), sb = pool_smem_bytes<LB, PAGES, WIDE>(G);
+    const int ma = pool_smem_bytes<LA, PAGES, WIDE>(DEC_GMAX), mb = pool_smem_bytes<LB, PAGES, WIDE>(DEC_GMAX);
+    const void *fn = reinterpret_cast<const void *>(decode_pool_kernel<LA, LB, ROT, PAGES, WIDE>);
     int nb = 1;
     if (prepare_kernel(fn, ma > mb ? ma : mb) != cudaSuccess ||
         kernel_occupancy(fn, DEC_WARPS * 32, sa > sb ? sa : sb, &nb) != cudaSuccess)
@@ -1058,49 +1166,40 @@ static auto dispatch_merged(int Lh, int Ll, F &f) {
   return f.template run<16, 8>();
 }
 
-template <bool ROT, bool PAGES>
+template <bool ROT, bool PAGES, bool WIDE>
 struct LaunchF {
   const DecParams &p;
   int grid;
   cudaStream_t st;
   template <int LA, int LB>
-  cudaError_t run() { return launch_pools<LA, LB, ROT, PAGES>(p, grid, st); }
+  cudaError_t run() { return launch_pools<LA, LB, ROT, PAGES, WIDE>(p, grid, st); }
 };
-template <bool ROT, bool PAGES>
+template <bool ROT, bool PAGES, bool WIDE>
 struct OccF {
   int G;
   template <int LA, int LB>
-  int run() { return pools_occupancy<LA, LB, ROT, PAGES>(G); }
+  int run() { return pools_occupancy<LA, LB, ROT, PAGES, WIDE>(G); }
 };
+
+// F<ROT, PAGES, WIDE> for the cache's layout, rotation and group size, built
+// from `args` and dispatched over the levels
+template <template <bool, bool, bool> class F, typename... A>
+static auto dispatch_cache(bool merged, int Lh, int Ll, const semkv_cache &c, A... args) {
+  const bool wide = c.H_q / c.H > 4;
+  auto go = [&](auto f) { return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(Lh, f); };
+  if (c.layout == SEMKV_LAYOUT_PAGES)
+    return wide ? go(F<false, true, true>{args...}) : go(F<false, true, false>{args...});
+  if (c.rotate) return go(F<true, false, false>{args...});       // rotation needs G <= 4
+  return wide ? go(F<false, false, true>{args...}) : go(F<false, false, false>{args...});
+}
 
 static cudaError_t launch_classes(bool merged, int Lh, int Ll, const semkv_cache &c, const DecParams &p, int grid,
                                   cudaStream_t st) {
-  const int L = Lh;
-  (void)Ll;
-  if (c.layout == SEMKV_LAYOUT_PAGES) {
-    LaunchF<false, true> f{p, grid, st};
-    return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(L, f);
-  }
-  if (c.rotate) {
-    LaunchF<true, false> f{p, grid, st};
-    return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(L, f);
-  }
-  LaunchF<false, false> f{p, grid, st};
-  return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(L, f);
+  return dispatch_cache<LaunchF>(merged, Lh, Ll, c, std::cref(p), grid, st);
 }
 
 static int class_occupancy(bool merged, int Lh, int Ll, const semkv_cache &c) {
-  const int G = c.H_q / c.H;
-  if (c.layout == SEMKV_LAYOUT_PAGES) {
-    OccF<false, true> f{G};
-    return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(Lh, f);
-  }
-  if (c.rotate) {
-    OccF<true, false> f{G};
-    return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(Lh, f);
-  }
-  OccF<false, false> f{G};
-  return merged ? dispatch_merged(Lh, Ll, f) : dispatch_one(Lh, f);
+  return dispatch_cache<OccF>(merged, Lh, Ll, c, c.H_q / c.H);
 }
 
 // code words of one slab of a class

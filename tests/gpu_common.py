@@ -74,5 +74,6 @@ def check_attention(out_gpu, out_ref):
     o = out_gpu.astype(np.float64)
     rel = np.linalg.norm(o - out_ref) / max(np.linalg.norm(out_ref), 1e-30)
     mx = np.max(np.abs(o - out_ref))
+    print(f"[attention error] rel-L2 {rel:.3e} max-abs {mx:.3e}")
     assert rel <= REL_L2 and mx <= MAX_ABS, (rel, mx)
     return rel, mx

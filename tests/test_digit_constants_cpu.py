@@ -83,3 +83,42 @@ def test_digit_chain_reproduces_base_L_digits(L):
     ref = [(np.arange(L ** k) // L ** s) % L for s in range(k)]
     for s in range(k):
         assert np.array_equal(digits[s], ref[s]), (L, s)
+
+
+@pytest.mark.parametrize("L", [L for L in range(3, 16) if L not in (4, 8)])
+def test_floor_chain_gives_every_floor_from_its_low_bits(L):
+    """The key side feeds the floors x_s = floor(P / L^s) of each part: x_0 is the
+    part's raw 16-bit field, and x_s (s >= 1) is the low 9 bits of the chain's t,
+    whose f16 pattern must be 0x6600 + x_s (t = 1536 + x_s with x_s < 512).  The
+    floors then give the digits as d_s = x_s - L x_(s+1) (x_k = 0)."""
+    parts, (c0, k0, c1, k1) = _plans()[L]
+    k = max(parts)
+    P = np.arange(L ** k, dtype=np.float64)
+    X = 1024 + P
+    c, K = _f16(c0), _f16(k0)
+    floors = [P.astype(np.int64)]
+    for s in range(1, k):
+        t = (X * c + K).astype(np.float16)
+        bits = t.view(np.uint16).astype(np.int64)
+        assert np.all((bits & 0xFE00) == 0x6600), (L, s)
+        floors.append(bits & 0x1FF)
+        X, c, K = t.astype(np.float64), _f16(c1), _f16(k1)
+    ints = np.arange(L ** k)
+    for s in range(k):
+        assert np.array_equal(floors[s], ints // L ** s), (L, s)
+    nxt = floors[1:] + [np.zeros_like(ints)]
+    for s in range(k):
+        assert np.array_equal(floors[s] - L * nxt[s], (ints // L ** s) % L), (L, s)
+
+
+def test_floor_coefficients_recover_the_digit_dot_product():
+    """sum_s q_s d_s over a part equals q_0 x_0 + sum_(s>=1) (q_s - L q_(s-1)) x_s:
+    the coefficients the key side's q fragments carry, checked on random parts."""
+    rng = np.random.default_rng(7)
+    for L, k in ((6, 3), (5, 4), (3, 5), (10, 3), (13, 2)):
+        q = rng.standard_normal(k)
+        coef = np.array([q[0]] + [q[s] - L * q[s - 1] for s in range(1, k)])
+        P = rng.integers(0, L ** k, 1000)
+        d = np.stack([(P // L ** s) % L for s in range(k)], 1)
+        x = np.stack([P // L ** s for s in range(k)], 1)
+        assert np.allclose(d @ q, x @ coef, rtol=0, atol=1e-9)
