@@ -385,19 +385,23 @@ __global__ void __launch_bounds__(AM_WARPS * 32, 1) attn_colsum_kernel(const Att
 }
 
 // ---- both passes on the 5th-generation tensor cores (tcgen05, TMEM accumulators)
-// CTA = (key chunk, KV head g, sequence b), 8 warps.  The Np <= 256 window rows
+// CTA = (key chunk, KV head g, sequence b), 16 warps.  The Np <= 256 window rows
 // of g's query heads stay in shared memory; 128-key tiles stream through a
 // 4-deep cp.async ring, all in the 128-byte-swizzled K-major layout the MMA
 // descriptors describe.  Thread 0 issues the MMAs of tile i into one of two
-// TMEM accumulators while the warps run the epilogue of tile i-1.
+// TMEM accumulators while the warps run the epilogue of tile i-1.  A warp
+// reads the TMEM lanes of its quadrant (warp % 4), so four warps share each
+// quadrant and split its columns.
 //   pass 1: D[rows][keys] = Q_g[rows] . K^T  (two M=128 halves of rows, N=128):
-//           each thread owns one row, keeps an online (max, sum of exp2) over
-//           its chunk, and writes one partial per (row, chunk);
+//           each thread owns one row and one 64-key half of every tile, keeps an
+//           online (max, sum of exp2) over its chunk, and writes one partial per
+//           (row, chunk, key half);
 //   pass 2: D[keys][rows] = K . Q_g^T  (M=128 keys, N=Np): each thread owns one
-//           key (warps w and w+4 split the rows) and sums exp2(s*c1 - M'_r),
-//           M'_r = M_r + log2(Z_r); one partial per (head, row half, key),
-//           summed in order by attn_headsum_kernel.
-constexpr int UA_THREADS = 256;
+//           key and one quarter of the rows (warps w, w+4, w+8, w+12) and sums
+//           exp2(s*c1 - M'_r), M'_r = M_r + log2(Z_r); one partial per (head,
+//           row quarter, key), summed in order by attn_headsum_kernel.
+constexpr int UA_THREADS = 512;
+constexpr int UA_RQ = 4;                          // pass-2 row quarters (head partials per key)
 constexpr int UA_KEYS = 128;
 constexpr int UA_MAXN = 256;
 constexpr int UA_NST = 4;                         // key tiles in the ring
@@ -421,7 +425,9 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int quarter = warp & 3, half = warp >> 2;
+  const int quarter = warp & 3;                    // TMEM lane quadrant of this warp
+  const int half = (warp >> 2) & 1, kh = warp >> 3; // pass 1: row half, key half of the tile
+  const int rq = warp >> 2;                        // pass 2: row quarter
   const int len = p.seq_len[b];
   if (len < 0 || len > p.T_max) return;            // flagged by the head-sum / merge kernels
   const int ntile = (len + UA_KEYS - 1) / UA_KEYS;
@@ -508,7 +514,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   const int row = half * 128 + quarter * 32 + lane;
   const int pos = (PASS == 1 && row < p.Rg) ? len - p.w + row % p.w : -1;
   float m_run = -INFINITY, l_run = 0.0f;
-  const int ncol_half = Np / 2;                    // pass 2: rows per warp half (Np is a multiple of 64)
+  const int ncol_q = Np / UA_RQ;                   // pass 2: rows per row quarter (a multiple of 16)
   bool lost = false;
   int nwait = 0;                                   // completed phases, per accumulator
   int pend = 0;                                    // accumulators with a commit not yet waited for
@@ -541,40 +547,42 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
       const bool edge = t0 + UA_KEYS - 1 > len - p.w;
       if (PASS == 1) {
         if (half * 128 < Np && !lost) {
-          const uint32_t la = tmem + ab * 256 + half * 128 + ((uint32_t)(quarter * 32) << 16);
-          // raw logits of this row for the 128 keys (c1 > 0: the max commutes with the scaling)
-          float v[128];
+          const uint32_t la = tmem + ab * 256 + half * 128 + kh * 64 + ((uint32_t)(quarter * 32) << 16);
+          // raw logits of this row for its 64 keys (c1 > 0: the max commutes with the scaling)
+          float v[64];
 #pragma unroll
-          for (int cb = 0; cb < 4; ++cb) tmem_ld32(la + cb * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[cb * 32]));
+          for (int cb = 0; cb < 2; ++cb) tmem_ld32(la + cb * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[cb * 32]));
           tmem_ld_wait();
           if (edge) {
-            const int lim = pos - t0;                // keys t0 + j with j > lim are masked
+            const int lim = pos - t0 - kh * 64;      // keys t0 + 64 kh + j with j > lim are masked
 #pragma unroll
-            for (int j = 0; j < 128; ++j) v[j] = j <= lim ? v[j] : -INFINITY;
+            for (int j = 0; j < 64; ++j) v[j] = j <= lim ? v[j] : -INFINITY;
           }
           float mr = v[0];
 #pragma unroll
-          for (int j = 1; j < 127; j += 2) mr = fmax3_nan(mr, v[j], v[j + 1]);
-          const float mx = fmax_nan(m_run, fmax_nan(mr, v[127]) * p.c1);
+          for (int j = 1; j < 63; j += 2) mr = fmax3_nan(mr, v[j], v[j + 1]);
+          const float mx = fmax_nan(m_run, fmax_nan(mr, v[63]) * p.c1);
           if (mx != -INFINITY) {
             float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-            for (int j = 0; j < 128; ++j) sum[j & 3] += ex2_approx(__fmaf_rn(v[j], p.c1, -mx));
+            for (int j = 0; j < 64; ++j) sum[j & 3] += ex2_approx(__fmaf_rn(v[j], p.c1, -mx));
             l_run = l_run * ex2_approx(m_run - mx) + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
             m_run = mx;
           }
         }
       } else {
         const int key = t0 + quarter * 32 + lane;
-        const int c0 = half * ncol_half;
+        const int c0 = rq * ncol_q;
         const uint32_t la = tmem + ab * 256 + c0 + ((uint32_t)(quarter * 32) << 16);
         float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        for (int cb = 0; cb < (lost ? 0 : ncol_half); cb += 64) {
+        for (int cb = 0; cb < (lost ? 0 : ncol_q); cb += 64) {
+          // (a load past the quarter reads columns of the next one, still inside
+          // the 256-column accumulator, and they are not used)
           uint32_t u[64];
           tmem_ld32(la + cb, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
           tmem_ld32(la + cb + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
           tmem_ld_wait();
-          const int nc = ncol_half - cb < 64 ? 32 : 64;   // ncol_half is a multiple of 32
+          const int nc = ncol_q - cb < 64 ? ncol_q - cb : 64;     // a multiple of 16
           if (!edge) {
             const float4 *M4 = reinterpret_cast<const float4 *>(Ms + c0 + cb);
 #pragma unroll
@@ -597,10 +605,10 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
           }
         }
         const float acc = (acc4[0] + acc4[1]) + (acc4[2] + acc4[3]);
-        // one partial per (KV head, column half, key): no exchange between the
-        // two warps of a key, the head-sum kernel adds the halves in order
+        // one partial per (KV head, row quarter, key): no exchange between the
+        // four warps of a key, the head-sum kernel adds the quarters in order
         if (key < p.T_max)
-          head_part[(((int64_t)b * p.H + g) * 2 + half) * p.T_max + key] = key < len ? acc : 0.0f;
+          head_part[(((int64_t)b * p.H + g) * UA_RQ + rq) * p.T_max + key] = key < len ? acc : 0.0f;
       }
       tc_fence_before();
     }
@@ -608,7 +616,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   if (PASS == 1) {
     if (half * 128 < Np && row < p.Rg) {
       const int hrow = (g * p.G + row / p.w) * p.w + row % p.w;    // h*w + i
-      p.part[((int64_t)b * p.H_q * p.w + hrow) * p.nchunk + chunk] = make_float2(m_run, l_run);
+      p.part[((int64_t)b * p.H_q * p.w + hrow) * p.nchunk + 2 * chunk + kh] = make_float2(m_run, l_run);
     }
   }
   cp_async_wait<0>();
@@ -637,7 +645,7 @@ __global__ void attn_headsum_kernel(const AttnParams p, const float *__restrict_
   }
   float s = 0.0f;
   if (j < len)
-    for (int g = 0; g < 2 * p.H; ++g) s += head_part[((int64_t)b * 2 * p.H + g) * p.T_max + j];
+    for (int g = 0; g < UA_RQ * p.H; ++g) s += head_part[((int64_t)b * UA_RQ * p.H + g) * p.T_max + j];
   p.score[idx] = s;
 }
 
@@ -646,7 +654,7 @@ size_t attn_mass_ws_bytes(int B, int T_max, int H, int H_q, int w) {
   const int ntile = (T_max + AM_TILE - 1) / AM_TILE;
   const int nchunk = ntile < 64 ? ntile : 64;
   const size_t parts = (size_t)(rows * nchunk * sizeof(float2) + rows * sizeof(float2) + 256);
-  return (parts + 255) / 256 * 256 + (size_t)B * H * 2 * T_max * sizeof(float) + 256;
+  return (parts + 255) / 256 * 256 + (size_t)B * H * UA_RQ * T_max * sizeof(float) + 256;
 }
 
 cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const uint16_t *q_win,
@@ -680,11 +688,12 @@ cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const u
   cudaError_t e;
   const int Np = (p.Rg + 63) / 64 * 64;       // two column halves of whole 32-column loads
   if (Np <= UA_MAXN) {
-    // tcgen05 path: one CTA per SM (all of TMEM), about one wave of CTAs
+    // tcgen05 path: one CTA per SM (all of TMEM), about one wave of CTAs;
+    // pass 1 writes two partials per (row, chunk), so at most 32 chunks
     const int utiles = (T_max + UA_KEYS - 1) / UA_KEYS;
     int nch = sms / (H * B);                  // whole waves only
-    nch = nch < 1 ? 1 : (nch > utiles ? utiles : (nch > 64 ? 64 : nch));
-    p.nchunk = nch;
+    nch = nch < 1 ? 1 : (nch > utiles ? utiles : (nch > 32 ? 32 : nch));
+    p.nchunk = 2 * nch;
     e = prepare_kernel(reinterpret_cast<const void *>(attn_umma_kernel<1>), UA_SMEM);
     if (e != cudaSuccess) return e;
     e = prepare_kernel(reinterpret_cast<const void *>(attn_umma_kernel<2>), UA_SMEM);
