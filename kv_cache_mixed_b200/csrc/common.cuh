@@ -131,6 +131,11 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
 }
 
 // max of three with NaN propagation (sm_100 three-input form)
+__device__ __forceinline__ float fmin3_nan(float a, float b, float c) {
+  float r;
+  asm("min.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 __device__ __forceinline__ float fmax3_nan(float a, float b, float c) {
   float r;
   asm("max.NaN.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -149,6 +154,11 @@ __device__ __forceinline__ void f2unpack(uint64_t v, float &lo, float &hi) {
 __device__ __forceinline__ uint64_t fma2_rn(uint64_t a, uint64_t b, uint64_t c) {
   uint64_t d;
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t mul2_rn(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
 __device__ __forceinline__ uint64_t add2_rn(uint64_t a, uint64_t b) {
