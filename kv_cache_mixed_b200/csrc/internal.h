@@ -1,6 +1,7 @@
 // internal.h -- host-side launchers shared by the C-ABI layer (not exported).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -18,6 +19,12 @@ int first_wait_polls(int dflt);
 int device_sm_count();
 cudaError_t prepare_kernel(const void *fn, int smem_bytes);
 cudaError_t kernel_occupancy(const void *fn, int threads, int smem_bytes, int *ctas_per_sm);
+// A tiled TMA descriptor over an fp16 tensor: dims fastest first, strides in
+// bytes of dims 1..rank-1, the box, and whether the box lands 128-byte
+// swizzled (the tensor cores' K-major operand layout).  Out-of-range elements
+// of a box read as zeros.
+cudaError_t encode_tensor_map_f16(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
+                                  const uint64_t *strides_bytes, const uint32_t *box, bool swizzle128);
 
 // Slot of each token within its class, and the high count per sequence.
 //   slot int32 [B][T_max], cnt_high int32 [B].

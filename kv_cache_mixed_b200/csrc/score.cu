@@ -15,6 +15,8 @@
 //   KV head run on tcgen05 with TMEM accumulators (attn_umma_kernel); wider
 //   groups on mma.sync m16n8k16.  Column sums are reduced in a fixed order, so
 //   the score is deterministic.
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 #include "umma.cuh"
@@ -410,15 +412,20 @@ constexpr int UA_KBYTES = UA_KEYS * 256;
 constexpr int UA_OFF_Q = 0;
 constexpr int UA_OFF_K = UA_QBYTES;
 constexpr int UA_OFF_M = UA_OFF_K + UA_NST * UA_KBYTES;          // float [256] M'_r (pass 2)
-constexpr int UA_OFF_BAR = UA_OFF_M + UA_MAXN * 4;                // u64 [2]
-constexpr int UA_OFF_SLOT = UA_OFF_BAR + 16;
+constexpr int UA_OFF_BAR = UA_OFF_M + UA_MAXN * 4;                // u64 [2] accumulators, [UA_NST] key tiles
+constexpr int UA_OFF_SLOT = UA_OFF_BAR + (2 + UA_NST) * 8;
 constexpr int UA_SMEM = UA_OFF_SLOT + 16 + 1024;
 constexpr int kUmmaWait = 1 << 22;
 static_assert(UA_OFF_K % 1024 == 0 && UA_KBYTES % 1024 == 0, "operand blocks must be 1024-byte aligned");
 
-template <int PASS>
+// TMA: the key tiles come in as two 128-byte-swizzled tensor boxes (dims 0..63
+// and 64..127 of 128 keys) issued by one thread and completing on the slot's
+// mbarrier; otherwise every thread stages 16-byte pieces with cp.async (keys
+// whose rows do not meet the tensor map's 16-byte stride rule).
+template <int PASS, bool TMA>
 __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnParams p, int Np, int nchunk,
-                                                                   float *head_part) {
+                                                                   float *head_part,
+                                                                   const __grid_constant__ CUtensorMap kmap) {
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment by an offset from the shared base, so that the compiler
   // still sees shared-memory pointers (plain shared loads, not generic ones)
@@ -438,9 +445,12 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   uint32_t *slot = reinterpret_cast<uint32_t *>(smem + UA_OFF_SLOT);
   const uint32_t sbase = smem_u32(smem);
   if (warp == 0) tmem_alloc(slot, 512);
+  uint64_t *tbars = bars + 2;                      // key tile slots (TMA)
   if (tid == 0) {
     mbar_init(&bars[0], 1);
     mbar_init(&bars[1], 1);
+#pragma unroll
+    for (int s = 0; s < UA_NST; ++s) mbar_init(&tbars[s], 1);
     fence_mbar_init();
   }
   // resident window rows of head g (zero past Rg), and pass 2's row constants
@@ -464,18 +474,35 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
     cp_async_commit();
   }
   const uint16_t *kg = p.k + (int64_t)b * p.kbs + (int64_t)g * p.T_max * kD;
+  uint32_t tpend = 0;                              // key slots with a TMA load not yet waited for
+  int tstaged[UA_NST];                             // (thread 0, TMA) the tile last loaded into each slot
   auto stage_keys = [&](int tile) {
     if (tile < te) {
-      uint8_t *kd = smem + UA_OFF_K + (tile % UA_NST) * UA_KBYTES;
+      const int sl = (tile - tb) % UA_NST;
+      uint8_t *kd = smem + UA_OFF_K + sl * UA_KBYTES;
       const int t0 = tile * UA_KEYS;
-      for (int i = tid; i < UA_KEYS * 16; i += UA_THREADS) {
-        const int r = i >> 4, c = i & 15;
-        const bool ok = t0 + r < p.T_max;
-        cp_async16_zfill(kd + sw128_offset(r, c, UA_KEYS), kg + (ok ? (int64_t)(t0 + r) * kD + c * 8 : 0), ok);
+      if constexpr (TMA) {
+        if (tid == 0) {
+          mbar_expect_tx(&tbars[sl], UA_KBYTES);
+          tma_load_4d(kd, &kmap, 0, t0, g, b, &tbars[sl]);
+          tma_load_4d(kd + UA_KEYS * 128, &kmap, 64, t0, g, b, &tbars[sl]);
+          tpend |= 1u << sl;
+          tstaged[sl] = tile;
+        }
+      } else {
+        for (int i = tid; i < UA_KEYS * 16; i += UA_THREADS) {
+          const int r = i >> 4, c = i & 15;
+          const bool ok = t0 + r < p.T_max;
+          cp_async16_zfill(kd + sw128_offset(r, c, UA_KEYS), kg + (ok ? (int64_t)(t0 + r) * kD + c * 8 : 0), ok);
+        }
       }
     }
-    cp_async_commit();
+    if constexpr (!TMA) cp_async_commit();
   };
+  if constexpr (TMA) {
+    cp_async_wait<0>();                            // the window rows
+    fence_proxy_async_smem();
+  }
   for (int i = 0; i < UA_NST - 2; ++i) stage_keys(tb + i);
 
   __syncthreads();
@@ -484,7 +511,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   const uint32_t qa = sbase + UA_OFF_Q;
 
   auto issue_mma = [&](int tile) {        // thread 0 only
-    const uint32_t ka = sbase + UA_OFF_K + (tile % UA_NST) * UA_KBYTES;
+    const uint32_t ka = sbase + UA_OFF_K + ((tile - tb) % UA_NST) * UA_KBYTES;
     const uint32_t acc = tmem + (tile & 1) * 256;
     if (PASS == 1) {
       const uint32_t idesc = umma_idesc_f16(128, UA_KEYS);
@@ -523,14 +550,26 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
     // issue tile `tile` (if any): its keys were staged two iterations ago
     if (tile < te) {
       stage_keys(tile + UA_NST - 2);               // slot of tile-2: its MMA was waited for last iteration
-      cp_async_wait<UA_NST - 2>();
-      fence_proxy_async_smem();
-      if (__syncthreads_or(lost)) break;           // an accumulator never arrived: stop issuing
-      if (tid == 0) {
-        tc_fence_after();
-        issue_mma(tile);
+      if constexpr (!TMA) {
+        cp_async_wait<UA_NST - 2>();
+        fence_proxy_async_smem();
       }
-      pend |= 1 << (tile & 1);
+      if (__syncthreads_or(lost)) break;           // an accumulator or a key tile never arrived: stop issuing
+      if (tid == 0) {
+        bool ok = true;
+        if constexpr (TMA) {
+          const int sl = (tile - tb) % UA_NST;
+          ok = mbar_wait(&tbars[sl], ((tile - tb) / UA_NST) & 1, kUmmaWait);
+          if (ok) tpend &= ~(1u << sl);
+        }
+        if (ok) {
+          tc_fence_after();
+          issue_mma(tile);
+        } else {
+          lost = true;
+        }
+      }
+      if (!(TMA && lost)) pend |= 1 << (tile & 1);
     }
     // epilogue of tile-1
     const int et = tile - 1;
@@ -623,10 +662,17 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   if (__syncthreads_or(lost) && tid == 0) {
     // drain: wait, with the full bound, for the commit of every accumulator
     // that still has MMAs in flight (the one whose wait gave up and the tile
-    // issued just before) before TMEM is freed
+    // issued just before) before TMEM is freed, and for every key tile load
+    // still in flight before the shared memory is released
     set_flag(p.status, SEMKV_FLAG_TIMEOUT);
     for (int ab = 0; ab < 2; ++ab)
       if (pend & (1 << ab)) mbar_wait(&bars[ab], (nwait >> ab) & 1, kUmmaWait);
+    if constexpr (TMA) {
+      // a slot's pending load is its latest tile; the phase parity is the
+      // number of earlier loads into that slot, mod 2
+      for (int sl = 0; sl < UA_NST; ++sl)
+        if ((tpend >> sl) & 1u) mbar_wait(&tbars[sl], ((tstaged[sl] - tb) / UA_NST) & 1, kUmmaWait);
+    }
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -694,17 +740,31 @@ cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const u
     int nch = sms / (H * B);                  // whole waves only
     nch = nch < 1 ? 1 : (nch > utiles ? utiles : (nch > 32 ? 32 : nch));
     p.nchunk = 2 * nch;
-    e = prepare_kernel(reinterpret_cast<const void *>(attn_umma_kernel<1>), UA_SMEM);
+    // keys [B][H][T_max][128] fp16 as a 4-D tensor map (dims fastest first),
+    // boxes of 64 dims x 128 keys landing 128-byte swizzled; it needs 16-byte
+    // aligned keys and a batch stride of whole 16-byte units
+    CUtensorMap kmap;
+    bool tma = (reinterpret_cast<uintptr_t>(k) & 15) == 0 && (k_bstride * 2) % 16 == 0;
+    if (tma) {
+      const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)T_max, (uint64_t)H, (uint64_t)B};
+      const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)T_max * kD * 2, (uint64_t)k_bstride * 2};
+      const uint32_t box[4] = {64, (uint32_t)UA_KEYS, 1, 1};
+      tma = encode_tensor_map_f16(&kmap, k, 4, dims, strides, box, true) == cudaSuccess;
+    }
+    if (!tma) memset(&kmap, 0, sizeof(kmap));
+    auto k1 = tma ? attn_umma_kernel<1, true> : attn_umma_kernel<1, false>;
+    auto k2 = tma ? attn_umma_kernel<2, true> : attn_umma_kernel<2, false>;
+    e = prepare_kernel(reinterpret_cast<const void *>(k1), UA_SMEM);
     if (e != cudaSuccess) return e;
-    e = prepare_kernel(reinterpret_cast<const void *>(attn_umma_kernel<2>), UA_SMEM);
+    e = prepare_kernel(reinterpret_cast<const void *>(k2), UA_SMEM);
     if (e != cudaSuccess) return e;
-    attn_umma_kernel<1><<<dim3(nch, H, B), UA_THREADS, UA_SMEM, st>>>(p, Np, nch, head_part);
+    k1<<<dim3(nch, H, B), UA_THREADS, UA_SMEM, st>>>(p, Np, nch, head_part, kmap);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_merge_kernel<<<(unsigned)((rows + 7) / 8), 256, 0, st>>>(p);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    attn_umma_kernel<2><<<dim3(nch, H, B), UA_THREADS, UA_SMEM, st>>>(p, Np, nch, head_part);
+    k2<<<dim3(nch, H, B), UA_THREADS, UA_SMEM, st>>>(p, Np, nch, head_part, kmap);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     attn_headsum_kernel<<<(unsigned)(((int64_t)B * T_max + 255) / 256), 256, 0, st>>>(p, head_part);
