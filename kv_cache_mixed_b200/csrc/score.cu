@@ -420,8 +420,9 @@ static_assert(UA_OFF_K % 1024 == 0 && UA_KBYTES % 1024 == 0, "operand blocks mus
 
 // TMA: the key tiles come in as two 128-byte-swizzled tensor boxes (dims 0..63
 // and 64..127 of 128 keys) issued by one thread and completing on the slot's
-// mbarrier; otherwise every thread stages 16-byte pieces with cp.async (keys
-// whose rows do not meet the tensor map's 16-byte stride rule).
+// mbarrier.  Otherwise every thread stages 16-byte pieces with cp.async: the
+// launcher takes that path only when the tensor map cannot be encoded (the
+// argument checks already guarantee the alignment it needs).
 template <int PASS, bool TMA>
 __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnParams p, int Np, int nchunk,
                                                                    float *head_part,
@@ -742,7 +743,8 @@ cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const u
     p.nchunk = 2 * nch;
     // keys [B][H][T_max][128] fp16 as a 4-D tensor map (dims fastest first),
     // boxes of 64 dims x 128 keys landing 128-byte swizzled; it needs 16-byte
-    // aligned keys and a batch stride of whole 16-byte units
+    // aligned keys and a batch stride of whole 16-byte units (both checked by
+    // semkv_score)
     CUtensorMap kmap;
     bool tma = (reinterpret_cast<uintptr_t>(k) & 15) == 0 && (k_bstride * 2) % 16 == 0;
     if (tma) {
