@@ -47,14 +47,16 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-# kernels one default step launches: attention-mass score 4 (row stats, merge,
-# column sums, head sum), select 1, quantize 3 (slot scan, quantize+pack, count
-# advance), append 1, decode 4 (one pool kernel per level, FP16 block, merge)
-LAUNCHES_PER_STEP = 4 + 1 + 3 + 1 + 4
-DECODE_LAUNCHES = 4
+# kernels one default step launches: attention-mass score 4 (pass 1, merge,
+# pass 2, head sum), select 1, quantize 3 (slot scan, quantize+pack, count
+# advance), append 1, decode 3 (both pools in one launch -- every level pair the
+# workloads use has a merged instance --, FP16 block, merge)
+LAUNCHES_PER_STEP = 4 + 1 + 3 + 1 + 3
+DECODE_LAUNCHES = 3
 QUANT_LAUNCHES = 3
 METRIC = "KV quantize+pack GB/s (FP16 in) & mixed-prec decode-attn GB/s vs HBM roofline"
 KERNEL_SOURCES = ["kv_cache_mixed_b200/csrc/quantize.cu", "kv_cache_mixed_b200/csrc/common.cuh"]
+DECODE_SOURCES = ["kv_cache_mixed_b200/csrc/decode.cu", "kv_cache_mixed_b200/csrc/common.cuh"]
 NOMINAL_HBM_GBS = 8000.0          # the 8 TB/s HBM3e figure the throughput target is stated against
 DEFAULT_WORKLOAD = "llama8b_prefill_T32768"
 WORKLOAD_NAMES = [DEFAULT_WORKLOAD, "llama8b_generation_B16", "mistral7b_T131072", "level_sweep_B8_T32768"]
@@ -224,16 +226,21 @@ def decode_algo_bytes(Lyr, H, H_q, B, nh_tokens, nl_tokens, Lh, Ll, buf_len):
             + 2 * B * Lyr * H * buf_len * 256 + 2 * B * Lyr * H_q * 128 * 2)
 
 
-def measured_traffic():
-    """Per-launch DRAM bytes of the quantize kernel from the committed ncu capture,
-    if it was taken on the current kernel sources (else None)."""
-    tp = os.path.join(ROOT, "profiles", "quantize_pack_traffic.json")
+def measured_traffic(record="quantize_pack_traffic.json", sources=None):
+    """Per-launch DRAM bytes of a kernel from its committed ncu capture record
+    (profiles/<record>), if it was taken on the current kernel sources (else None)."""
+    tp = os.path.join(ROOT, "profiles", record)
     if not os.path.exists(tp):
         return None
     import hashlib
     d = json.load(open(tp))
-    hsh = hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read() for f in KERNEL_SOURCES)).hexdigest()
+    hsh = hashlib.sha256(b"".join(open(os.path.join(ROOT, f), "rb").read()
+                                  for f in (sources or KERNEL_SOURCES))).hexdigest()
     return d.get("dram_bytes_per_launch") if d.get("source_sha256") == hsh else None
+
+
+def measured_decode_traffic():
+    return measured_traffic("decode_pool_traffic.json", DECODE_SOURCES)
 
 
 def cpu_cores_used(fn):
@@ -342,8 +349,8 @@ def run_prefill(args, rank, world, dist):
     q_ms, d_ms = stage["quantize"], stage["decode"]
     rq = roofline("quantize_pack_kernel (+ slot scan and count kernels of semkv_quantize)", quant_bytes, q_ms,
                   measured_traffic())
-    rd = roofline("decode_pool_kernel x2 + decode_buffer_kernel + decode_merge_kernel (semkv_decode_attn)",
-                  dec_bytes, d_ms)
+    rd = roofline("decode_pool_kernel (both pools) + decode_buffer_kernel + decode_merge_kernel (semkv_decode_attn)",
+                  dec_bytes, d_ms, measured_decode_traffic())
     value = job_value(world, fp16_in, ms)
     res = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -572,7 +579,7 @@ def run_generation(args, rank, world, dist):
                                         wl.L_high, wl.L_low, buf_lens[s]))
     dec_gbs = sum(dbytes) / (dec.sum() * 1e-3) / 1e9
     fl = np.array(flush)
-    rd = roofline("semkv_decode_attn (2 pool kernels, FP16-block kernel, merge), one generation step",
+    rd = roofline("semkv_decode_attn (both pools in one kernel, FP16-block kernel, merge), one generation step",
                   float(np.mean(dbytes)), float(dec.mean()))
     quant_bytes = quant_algo_bytes(B, Lyr, H, prompt_tokens, nh_tok, nl_tok, wl.L_high, wl.L_low, T)
     rq = roofline("quantize_pack_kernel of the prompt (+ slot scan and counts)", quant_bytes, qms)
