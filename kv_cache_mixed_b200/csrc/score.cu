@@ -15,8 +15,6 @@
 //   KV head run on tcgen05 with TMEM accumulators (attn_umma_kernel); wider
 //   groups on mma.sync m16n8k16.  Column sums are reduced in a fixed order, so
 //   the score is deterministic.
-#include <cstring>
-
 #include "common.cuh"
 #include "internal.h"
 #include "umma.cuh"
@@ -387,13 +385,16 @@ __global__ void __launch_bounds__(AM_WARPS * 32, 1) attn_colsum_kernel(const Att
 }
 
 // ---- both passes on the 5th-generation tensor cores (tcgen05, TMEM accumulators)
-// CTA = (key chunk, KV head g, sequence b), 16 warps.  The Np <= 256 window rows
-// of g's query heads stay in shared memory; 128-key tiles stream through a
-// 4-deep cp.async ring, all in the 128-byte-swizzled K-major layout the MMA
-// descriptors describe.  Thread 0 issues the MMAs of tile i into one of two
-// TMEM accumulators while the warps run the epilogue of tile i-1.  A warp
-// reads the TMEM lanes of its quadrant (warp % 4), so four warps share each
-// quadrant and split its columns.
+// CTA = (key chunk, KV head g, sequence b): 16 epilogue warps and one producer
+// warp.  The Np <= 256 window rows of g's query heads stay in shared memory.
+// The producer's lane 0 loads the 128-key tiles as two 128-byte-swizzled TMA
+// tensor boxes (dims 0..63 and 64..127) into a 4-slot ring and issues each
+// tile's MMAs into one of two TMEM accumulators (tile i into accumulator i%2,
+// once the epilogue warps have released it).  Each epilogue warp waits for the
+// tile's accumulator, reads its TMEM lanes (quadrant warp % 4) and releases the
+// accumulator with one arrival: no CTA-wide barrier per tile, so a warp runs on
+// to the next tile as soon as its MMAs are done, and the warps' exp2 bursts
+// spread out instead of meeting.
 //   pass 1: D[rows][keys] = Q_g[rows] . K^T  (two M=128 halves of rows, N=128):
 //           each thread owns one row and one 64-key half of every tile, keeps an
 //           online (max, sum of exp2) over its chunk, and writes one partial per
@@ -402,7 +403,8 @@ __global__ void __launch_bounds__(AM_WARPS * 32, 1) attn_colsum_kernel(const Att
 //           key and one quarter of the rows (warps w, w+4, w+8, w+12) and sums
 //           exp2(s*c1 - M'_r), M'_r = M_r + log2(Z_r); one partial per (head,
 //           row quarter, key), summed in order by attn_headsum_kernel.
-constexpr int UA_THREADS = 512;
+constexpr int UA_EPI_WARPS = 16;
+constexpr int UA_THREADS = (UA_EPI_WARPS + 1) * 32;   // + the producer warp
 constexpr int UA_RQ = 4;                          // pass-2 row quarters (head partials per key)
 constexpr int UA_KEYS = 128;
 constexpr int UA_MAXN = 256;
@@ -412,18 +414,19 @@ constexpr int UA_KBYTES = UA_KEYS * 256;
 constexpr int UA_OFF_Q = 0;
 constexpr int UA_OFF_K = UA_QBYTES;
 constexpr int UA_OFF_M = UA_OFF_K + UA_NST * UA_KBYTES;          // float [256] M'_r (pass 2)
-constexpr int UA_OFF_BAR = UA_OFF_M + UA_MAXN * 4;                // u64 [2] accumulators, [UA_NST] key tiles
-constexpr int UA_OFF_SLOT = UA_OFF_BAR + (2 + UA_NST) * 8;
+// mbarriers: [2] accumulator full (MMA commit), [2] accumulator free (16 warp
+// arrivals), [UA_NST] key tile landed (TMA)
+constexpr int UA_OFF_BAR = UA_OFF_M + UA_MAXN * 4;
+constexpr int UA_OFF_SLOT = UA_OFF_BAR + (4 + UA_NST) * 8;
 constexpr int UA_SMEM = UA_OFF_SLOT + 16 + 1024;
 constexpr int kUmmaWait = 1 << 22;
 static_assert(UA_OFF_K % 1024 == 0 && UA_KBYTES % 1024 == 0, "operand blocks must be 1024-byte aligned");
 
-// TMA: the key tiles come in as two 128-byte-swizzled tensor boxes (dims 0..63
-// and 64..127 of 128 keys) issued by one thread and completing on the slot's
-// mbarrier.  Otherwise every thread stages 16-byte pieces with cp.async: the
-// launcher takes that path only when the tensor map cannot be encoded (the
-// argument checks already guarantee the alignment it needs).
-template <int PASS, bool TMA>
+__device__ __forceinline__ void mbar_arrive_one(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
+template <int PASS>
 __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnParams p, int Np, int nchunk,
                                                                    float *head_part,
                                                                    const __grid_constant__ CUtensorMap kmap) {
@@ -433,6 +436,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = warp == UA_EPI_WARPS;
   const int quarter = warp & 3;                    // TMEM lane quadrant of this warp
   const int half = (warp >> 2) & 1, kh = warp >> 3; // pass 1: row half, key half of the tile
   const int rq = warp >> 2;                        // pass 2: row quarter
@@ -440,16 +444,20 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
   if (len < 0 || len > p.T_max) return;            // flagged by the head-sum / merge kernels
   const int ntile = (len + UA_KEYS - 1) / UA_KEYS;
   const int tb = (int)((int64_t)ntile * chunk / nchunk), te = (int)((int64_t)ntile * (chunk + 1) / nchunk);
+  const int n = te - tb;                           // this CTA's tiles; local tile i = tb + i
 
   float *Ms = reinterpret_cast<float *>(smem + UA_OFF_M);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + UA_OFF_BAR);
+  uint64_t *full = reinterpret_cast<uint64_t *>(smem + UA_OFF_BAR);    // [2]
+  uint64_t *freeb = full + 2;                                           // [2]
+  uint64_t *tbars = full + 4;                                           // [UA_NST]
   uint32_t *slot = reinterpret_cast<uint32_t *>(smem + UA_OFF_SLOT);
   const uint32_t sbase = smem_u32(smem);
   if (warp == 0) tmem_alloc(slot, 512);
-  uint64_t *tbars = bars + 2;                      // key tile slots (TMA)
   if (tid == 0) {
-    mbar_init(&bars[0], 1);
-    mbar_init(&bars[1], 1);
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    mbar_init(&freeb[0], UA_EPI_WARPS);
+    mbar_init(&freeb[1], UA_EPI_WARPS);
 #pragma unroll
     for (int s = 0; s < UA_NST; ++s) mbar_init(&tbars[s], 1);
     fence_mbar_init();
@@ -473,120 +481,100 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
       }
     }
     cp_async_commit();
+    cp_async_wait<0>();
+    fence_proxy_async_smem();                      // the window rows feed the tensor cores
   }
-  const uint16_t *kg = p.k + (int64_t)b * p.kbs + (int64_t)g * p.T_max * kD;
-  uint32_t tpend = 0;                              // key slots with a TMA load not yet waited for
-  int tstaged[UA_NST];                             // (thread 0, TMA) the tile last loaded into each slot
-  auto stage_keys = [&](int tile) {
-    if (tile < te) {
-      const int sl = (tile - tb) % UA_NST;
-      uint8_t *kd = smem + UA_OFF_K + sl * UA_KBYTES;
-      const int t0 = tile * UA_KEYS;
-      if constexpr (TMA) {
-        if (tid == 0) {
-          mbar_expect_tx(&tbars[sl], UA_KBYTES);
-          tma_load_4d(kd, &kmap, 0, t0, g, b, &tbars[sl]);
-          tma_load_4d(kd + UA_KEYS * 128, &kmap, 64, t0, g, b, &tbars[sl]);
-          tpend |= 1u << sl;
-          tstaged[sl] = tile;
-        }
-      } else {
-        for (int i = tid; i < UA_KEYS * 16; i += UA_THREADS) {
-          const int r = i >> 4, c = i & 15;
-          const bool ok = t0 + r < p.T_max;
-          cp_async16_zfill(kd + sw128_offset(r, c, UA_KEYS), kg + (ok ? (int64_t)(t0 + r) * kD + c * 8 : 0), ok);
-        }
-      }
-    }
-    if constexpr (!TMA) cp_async_commit();
-  };
-  if constexpr (TMA) {
-    cp_async_wait<0>();                            // the window rows
-    fence_proxy_async_smem();
-  }
-  for (int i = 0; i < UA_NST - 2; ++i) stage_keys(tb + i);
-
   __syncthreads();
   const uint32_t tmem = *slot;
   tc_fence_after();
   const uint32_t qa = sbase + UA_OFF_Q;
-
-  auto issue_mma = [&](int tile) {        // thread 0 only
-    const uint32_t ka = sbase + UA_OFF_K + ((tile - tb) % UA_NST) * UA_KBYTES;
-    const uint32_t acc = tmem + (tile & 1) * 256;
-    if (PASS == 1) {
-      const uint32_t idesc = umma_idesc_f16(128, UA_KEYS);
-      for (int hf = 0; hf * 128 < Np; ++hf) {
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t off = (ks & 3) * 32;
-          const uint64_t adesc = umma_desc_sw128(qa + (ks >> 2) * (Np * 128) + hf * 128 * 128 + off);
-          const uint64_t bdesc = umma_desc_sw128(ka + (ks >> 2) * (UA_KEYS * 128) + off);
-          umma_f16(acc + hf * 128, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
-        }
-      }
-    } else {
-      const uint32_t idesc = umma_idesc_f16(UA_KEYS, Np);
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint32_t off = (ks & 3) * 32;
-        const uint64_t adesc = umma_desc_sw128(ka + (ks >> 2) * (UA_KEYS * 128) + off);
-        const uint64_t bdesc = umma_desc_sw128(qa + (ks >> 2) * (Np * 128) + off);
-        umma_f16(acc, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
-      }
-    }
-    umma_commit(&bars[tile & 1]);
-  };
-
-  // pass 1 state: this thread's row; pass 2: this thread's key and column half
-  const int row = half * 128 + quarter * 32 + lane;
-  const int pos = (PASS == 1 && row < p.Rg) ? len - p.w + row % p.w : -1;
-  float m_run = -INFINITY, l_run = 0.0f;
-  const int ncol_q = Np / UA_RQ;                   // pass 2: rows per row quarter (a multiple of 16)
   bool lost = false;
-  int nwait = 0;                                   // completed phases, per accumulator
-  int pend = 0;                                    // accumulators with a commit not yet waited for
 
-  for (int tile = tb; tile <= te; ++tile) {
-    // issue tile `tile` (if any): its keys were staged two iterations ago
-    if (tile < te) {
-      stage_keys(tile + UA_NST - 2);               // slot of tile-2: its MMA was waited for last iteration
-      if constexpr (!TMA) {
-        cp_async_wait<UA_NST - 2>();
-        fence_proxy_async_smem();
-      }
-      if (__syncthreads_or(lost)) break;           // an accumulator or a key tile never arrived: stop issuing
-      if (tid == 0) {
-        bool ok = true;
-        if constexpr (TMA) {
-          const int sl = (tile - tb) % UA_NST;
-          ok = mbar_wait(&tbars[sl], ((tile - tb) / UA_NST) & 1, kUmmaWait);
-          if (ok) tpend &= ~(1u << sl);
+  if (producer) {
+    if (lane == 0) {
+      uint32_t tpend = 0;                          // slots with a load in flight
+      int tstaged[UA_NST];                         // the local tile last loaded into each slot
+      auto stage = [&](int i) {                    // local tile i into slot i % UA_NST
+        if (i < n) {
+          const int sl = i % UA_NST;
+          uint8_t *kd = smem + UA_OFF_K + sl * UA_KBYTES;
+          const int t0 = (tb + i) * UA_KEYS;
+          mbar_expect_tx(&tbars[sl], UA_KBYTES);
+          tma_load_4d(kd, &kmap, 0, t0, g, b, &tbars[sl]);
+          tma_load_4d(kd + UA_KEYS * 128, &kmap, 64, t0, g, b, &tbars[sl]);
+          tpend |= 1u << sl;
+          tstaged[sl] = i;
         }
-        if (ok) {
-          tc_fence_after();
-          issue_mma(tile);
+      };
+      for (int i = 0; i < UA_NST; ++i) stage(i);
+      int issued = 0;                              // MMAs issued (local tiles 0 .. issued-1)
+      for (int i = 0; i < n; ++i) {
+        const int sl = i % UA_NST, ab = i & 1;
+        // the tile's keys have landed, and the accumulator's last tile (i-2)
+        // has been read by all 16 epilogue warps
+        if (!mbar_wait(&tbars[sl], (i / UA_NST) & 1, kUmmaWait)) { lost = true; break; }
+        tpend &= ~(1u << sl);
+        if (i >= 2 && !mbar_wait(&freeb[ab], ((i - 2) >> 1) & 1, kUmmaWait)) { lost = true; break; }
+        tc_fence_after();
+        const uint32_t ka = sbase + UA_OFF_K + sl * UA_KBYTES;
+        const uint32_t acc = tmem + ab * 256;
+        if (PASS == 1) {
+          const uint32_t idesc = umma_idesc_f16(128, UA_KEYS);
+          for (int hf = 0; hf * 128 < Np; ++hf) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint32_t off = (ks & 3) * 32;
+              const uint64_t adesc = umma_desc_sw128(qa + (ks >> 2) * (Np * 128) + hf * 128 * 128 + off);
+              const uint64_t bdesc = umma_desc_sw128(ka + (ks >> 2) * (UA_KEYS * 128) + off);
+              umma_f16(acc + hf * 128, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+            }
+          }
         } else {
-          lost = true;
+          const uint32_t idesc = umma_idesc_f16(UA_KEYS, Np);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t off = (ks & 3) * 32;
+            const uint64_t adesc = umma_desc_sw128(ka + (ks >> 2) * (UA_KEYS * 128) + off);
+            const uint64_t bdesc = umma_desc_sw128(qa + (ks >> 2) * (Np * 128) + off);
+            umma_f16(acc, adesc, bdesc, idesc, ks > 0 ? 1u : 0u);
+          }
+        }
+        umma_commit(&full[ab]);
+        issued = i + 1;
+        // the slot of tile i-1 is free once its MMAs are done: load tile i+3 there
+        if (i >= 1) {
+          if (!mbar_wait(&full[(i - 1) & 1], ((i - 1) >> 1) & 1, kUmmaWait)) { lost = true; break; }
+          stage(i - 1 + UA_NST);
         }
       }
-      if (!(TMA && lost)) pend |= 1 << (tile & 1);
+      if (lost) {
+        // drain: wait, with the full bound, for the commits of the MMAs issued
+        // (the last two) and for every key tile load still in flight, before
+        // TMEM and shared memory are freed
+        set_flag(p.status, SEMKV_FLAG_TIMEOUT);
+        for (int i = issued - 2 < 0 ? 0 : issued - 2; i < issued; ++i)
+          mbar_wait(&full[i & 1], (i >> 1) & 1, kUmmaWait);
+        for (int sl = 0; sl < UA_NST; ++sl)
+          if ((tpend >> sl) & 1u) mbar_wait(&tbars[sl], (tstaged[sl] / UA_NST) & 1, kUmmaWait);
+      }
     }
-    // epilogue of tile-1
-    const int et = tile - 1;
-    if (et >= tb) {
-      const int ab = et & 1;
-      if (mbar_wait(&bars[ab], (nwait >> ab) & 1, kUmmaWait)) {
-        nwait ^= 1 << ab;
-        pend &= ~(1 << ab);
-      } else {
+  } else {
+    // epilogue warps
+    const int row = half * 128 + quarter * 32 + lane;
+    const int pos = (PASS == 1 && row < p.Rg) ? len - p.w + row % p.w : -1;
+    float m_run = -INFINITY, l_run = 0.0f;
+    const int ncol_q = Np / UA_RQ;                 // pass 2: rows per row quarter (a multiple of 16)
+    for (int i = 0; i < n; ++i) {
+      const int ab = i & 1;
+      if (!mbar_wait(&full[ab], (i >> 1) & 1, kUmmaWait)) {
         lost = true;
+        break;
       }
       tc_fence_after();
-      const int t0 = et * UA_KEYS;
+      const int t0 = (tb + i) * UA_KEYS;
       const bool edge = t0 + UA_KEYS - 1 > len - p.w;
       if (PASS == 1) {
-        if (half * 128 < Np && !lost) {
+        if (half * 128 < Np) {
           const uint32_t la = tmem + ab * 256 + half * 128 + kh * 64 + ((uint32_t)(quarter * 32) << 16);
           // raw logits of this row for its 64 keys (c1 > 0: the max commutes with the scaling)
           float v[64];
@@ -615,7 +603,7 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
         const int c0 = rq * ncol_q;
         const uint32_t la = tmem + ab * 256 + c0 + ((uint32_t)(quarter * 32) << 16);
         float acc4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-        for (int cb = 0; cb < (lost ? 0 : ncol_q); cb += 64) {
+        for (int cb = 0; cb < ncol_q; cb += 64) {
           // (a load past the quarter reads columns of the next one, still inside
           // the 256-column accumulator, and they are not used)
           uint32_t u[64];
@@ -651,29 +639,16 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
           head_part[(((int64_t)b * p.H + g) * UA_RQ + rq) * p.T_max + key] = key < len ? acc : 0.0f;
       }
       tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_one(&freeb[ab]);   // this warp is done with the accumulator
     }
-  }
-  if (PASS == 1) {
-    if (half * 128 < Np && row < p.Rg) {
-      const int hrow = (g * p.G + row / p.w) * p.w + row % p.w;    // h*w + i
-      p.part[((int64_t)b * p.H_q * p.w + hrow) * p.nchunk + 2 * chunk + kh] = make_float2(m_run, l_run);
+    if (PASS == 1) {
+      if (half * 128 < Np && row < p.Rg) {
+        const int hrow = (g * p.G + row / p.w) * p.w + row % p.w;    // h*w + i
+        p.part[((int64_t)b * p.H_q * p.w + hrow) * p.nchunk + 2 * chunk + kh] = make_float2(m_run, l_run);
+      }
     }
-  }
-  cp_async_wait<0>();
-  if (__syncthreads_or(lost) && tid == 0) {
-    // drain: wait, with the full bound, for the commit of every accumulator
-    // that still has MMAs in flight (the one whose wait gave up and the tile
-    // issued just before) before TMEM is freed, and for every key tile load
-    // still in flight before the shared memory is released
-    set_flag(p.status, SEMKV_FLAG_TIMEOUT);
-    for (int ab = 0; ab < 2; ++ab)
-      if (pend & (1 << ab)) mbar_wait(&bars[ab], (nwait >> ab) & 1, kUmmaWait);
-    if constexpr (TMA) {
-      // a slot's pending load is its latest tile; the phase parity is the
-      // number of earlier loads into that slot, mod 2
-      for (int sl = 0; sl < UA_NST; ++sl)
-        if ((tpend >> sl) & 1u) mbar_wait(&tbars[sl], ((tstaged[sl] - tb) / UA_NST) & 1, kUmmaWait);
-    }
+    if (lost && lane == 0) set_flag(p.status, SEMKV_FLAG_TIMEOUT);
   }
   __syncthreads();
   if (warp == 0) tmem_dealloc(tmem, 512);
@@ -746,16 +721,15 @@ cudaError_t launch_score_attn_mass(const uint16_t *k, int64_t k_bstride, const u
     // aligned keys and a batch stride of whole 16-byte units (both checked by
     // semkv_score)
     CUtensorMap kmap;
-    bool tma = (reinterpret_cast<uintptr_t>(k) & 15) == 0 && (k_bstride * 2) % 16 == 0;
-    if (tma) {
+    {
       const uint64_t dims[4] = {(uint64_t)kD, (uint64_t)T_max, (uint64_t)H, (uint64_t)B};
       const uint64_t strides[3] = {(uint64_t)kD * 2, (uint64_t)T_max * kD * 2, (uint64_t)k_bstride * 2};
       const uint32_t box[4] = {64, (uint32_t)UA_KEYS, 1, 1};
-      tma = encode_tensor_map_f16(&kmap, k, 4, dims, strides, box, true) == cudaSuccess;
+      e = encode_tensor_map_f16(&kmap, k, 4, dims, strides, box, true);
+      if (e != cudaSuccess) return e;
     }
-    if (!tma) memset(&kmap, 0, sizeof(kmap));
-    auto k1 = tma ? attn_umma_kernel<1, true> : attn_umma_kernel<1, false>;
-    auto k2 = tma ? attn_umma_kernel<2, true> : attn_umma_kernel<2, false>;
+    auto k1 = attn_umma_kernel<1>;
+    auto k2 = attn_umma_kernel<2>;
     e = prepare_kernel(reinterpret_cast<const void *>(k1), UA_SMEM);
     if (e != cudaSuccess) return e;
     e = prepare_kernel(reinterpret_cast<const void *>(k2), UA_SMEM);
