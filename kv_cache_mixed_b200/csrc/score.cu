@@ -586,16 +586,22 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
 #pragma unroll
             for (int j = 0; j < 64; ++j) v[j] = j <= lim ? v[j] : -INFINITY;
           }
-          float mr = v[0];
+          // two 32-key halves, each an online update: the max of the second half
+          // is independent of the first half's exp2, so the two interleave
 #pragma unroll
-          for (int j = 1; j < 63; j += 2) mr = fmax3_nan(mr, v[j], v[j + 1]);
-          const float mx = fmax_nan(m_run, fmax_nan(mr, v[63]) * p.c1);
-          if (mx != -INFINITY) {
-            float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+          for (int hk = 0; hk < 2; ++hk) {
+            const float *vh = v + 32 * hk;
+            float mr = vh[0];
 #pragma unroll
-            for (int j = 0; j < 64; ++j) sum[j & 3] += ex2_approx(__fmaf_rn(v[j], p.c1, -mx));
-            l_run = l_run * ex2_approx(m_run - mx) + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
-            m_run = mx;
+            for (int j = 1; j < 31; j += 2) mr = fmax3_nan(mr, vh[j], vh[j + 1]);
+            const float mx = fmax_nan(m_run, fmax_nan(mr, vh[31]) * p.c1);
+            if (mx != -INFINITY) {
+              float sum[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+              for (int j = 0; j < 32; ++j) sum[j & 3] += ex2_approx(__fmaf_rn(vh[j], p.c1, -mx));
+              l_run = l_run * ex2_approx(m_run - mx) + ((sum[0] + sum[1]) + (sum[2] + sum[3]));
+              m_run = mx;
+            }
           }
         }
       } else {
@@ -613,14 +619,22 @@ __global__ void __launch_bounds__(UA_THREADS, 1) attn_umma_kernel(const AttnPara
           const int nc = ncol_q - cb < 64 ? ncol_q - cb : 64;     // a multiple of 16
           if (!edge) {
             const float4 *M4 = reinterpret_cast<const float4 *>(Ms + c0 + cb);
-#pragma unroll
-            for (int j4 = 0; j4 < 16; ++j4) {
-              if (j4 * 4 >= nc) break;
+            auto col4 = [&](int j4) {
               const float4 m4 = M4[j4];
               acc4[0] += ex2_approx(__fmaf_rn(__uint_as_float(u[4 * j4 + 0]), p.c1, -m4.x));
               acc4[1] += ex2_approx(__fmaf_rn(__uint_as_float(u[4 * j4 + 1]), p.c1, -m4.y));
               acc4[2] += ex2_approx(__fmaf_rn(__uint_as_float(u[4 * j4 + 2]), p.c1, -m4.z));
               acc4[3] += ex2_approx(__fmaf_rn(__uint_as_float(u[4 * j4 + 3]), p.c1, -m4.w));
+            };
+            if (nc == 64) {
+#pragma unroll
+              for (int j4 = 0; j4 < 16; ++j4) col4(j4);
+            } else {
+#pragma unroll
+              for (int j4 = 0; j4 < 16; ++j4) {
+                if (j4 * 4 >= nc) break;
+                col4(j4);
+              }
             }
           } else {
 #pragma unroll
@@ -666,8 +680,19 @@ __global__ void attn_headsum_kernel(const AttnParams p, const float *__restrict_
     return;
   }
   float s = 0.0f;
-  if (j < len)
-    for (int g = 0; g < UA_RQ * p.H; ++g) s += head_part[((int64_t)b * UA_RQ * p.H + g) * p.T_max + j];
+  if (j < len) {
+    // the partials in order; eight loads in flight before they are added
+    const int np = UA_RQ * p.H;
+    const float *hp = head_part + (int64_t)b * np * p.T_max + j;
+    for (int g0 = 0; g0 < np; g0 += 8) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = g0 + i < np ? __ldg(hp + (int64_t)(g0 + i) * p.T_max) : 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (g0 + i < np) s += v[i];
+    }
+  }
   p.score[idx] = s;
 }
 
