@@ -72,7 +72,8 @@ def parse(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-options", action="store_true", help="skip the option timings (score accumulation, rotation)")
-    ap.add_argument("--case", default=None, choices=["score", "select", "quantize", "decode"],
+    ap.add_argument("--case", default=None, choices=["score", "select", "quantize", "decode", "quantize_rotated",
+                                                     "quantize_pages"],
                     help="profiling case: run only this stage, on the prefill workload cut to --layers layers")
     ap.add_argument("--layers", type=int, default=4)
     return ap.parse_args(argv)
@@ -873,7 +874,8 @@ def run_case(args):
     mask = torch.empty((B, T), dtype=torch.uint8, device=dev)
     out = torch.empty_like(qdec)
     nh = kv.semkv_num_high(T, wl.r_ppm)
-    cache = kv.MixedCache(B, Lyr, H, H_q, wl.L_high, wl.L_low, wl.r_ppm, nh + 128, T - nh + 128)
+    opts = {"quantize_rotated": {"rotate": True}, "quantize_pages": {"layout": kv.LAYOUT_PAGES}}.get(args.case, {})
+    cache = kv.MixedCache(B, Lyr, H, H_q, wl.L_high, wl.L_low, wl.r_ppm, nh + 128, T - nh + 128, **opts)
     kv.semkv_score(kv.SCORE_ATTN_MASS, k[:, Lyr - 1], k.stride(0), q_win, seq_len, B, T, H, H_q, w, score)
     kv.semkv_select(score, seq_len, wl.r_ppm, mask)
     kv.semkv_quantize(cache, k, v, seq_len, mask)
@@ -887,7 +889,7 @@ def run_case(args):
             kv.semkv_score(kv.SCORE_ATTN_MASS, k[:, Lyr - 1], k.stride(0), q_win, seq_len, B, T, H, H_q, w, score)
         elif args.case == "select":
             kv.semkv_select(score, seq_len, wl.r_ppm, mask)
-        elif args.case == "quantize":
+        elif args.case.startswith("quantize"):
             cache.n_high.zero_()
             cache.n_low.zero_()
             kv.semkv_quantize(cache, k, v, seq_len, mask)
