@@ -164,6 +164,21 @@ const char *semkv_version(void);
  */
 void semkv_set_first_copy_wait_polls(int32_t polls);
 
+/*
+ * Self-check of the reciprocal the quantizer uses (no counterpart on the
+ * pages).  Quantize forms a row's r = RN(1/scale) from the hardware's
+ * approximate reciprocal and one Newton-Raphson step in fused multiply-adds,
+ * not from an IEEE divide.  This call compares that reciprocal bit for bit with
+ * the IEEE round-to-nearest reciprocal for every positive float whose exponent
+ * field lies in [exp_lo, exp_hi] (2^23 values per exponent), and adds the
+ * number of differences to *mismatches (device, unsigned 64-bit, caller
+ * zeroed), enqueued on `stream`.  Exponent fields 1 .. 252 (b in [2^-126,
+ * 2^126)) cover every scale a row can have, and there the count must be 0.
+ * INVALID_ARG for exp_lo < 1, exp_hi > 254, exp_lo > exp_hi or a null pointer.
+ */
+semkv_status semkv_check_reciprocal(uint32_t exp_lo, uint32_t exp_hi, unsigned long long *mismatches,
+                                    void *stream);
+
 /* ---- a1: importance score (Fig. 2) ---------------------------------------- */
 
 /* Workspace bytes semkv_score needs for these sizes (0 for KEY_L2). */

@@ -9,5 +9,5 @@ from .binding import (FLAG_CAPACITY, FLAG_NONFINITE, FLAG_SEQLEN, FLAG_TIMEOUT, 
                       SCORE_KEY_L2, EXPORTED, LIB_PATH, MixedCache, SemkvError, semkv_append_block,
                       semkv_decode_attn, semkv_decode_attn_acc, semkv_digits_per_word, semkv_num_high, semkv_quantize,
                       semkv_quantize_noalloc, semkv_score, semkv_select, semkv_set_first_copy_wait_polls,
-                      semkv_version,
+                      semkv_check_reciprocal, semkv_version,
                       semkv_words_per_row)

@@ -54,6 +54,7 @@ _lib_row_bits = _sig("semkv_row_bits", _i32, [_i32, _i32])
 _lib_pool_words = _sig("semkv_pool_words", _i64, [_i32, _i32, _i32])
 _lib_version = _sig("semkv_version", ctypes.c_char_p, [])
 _lib_set_wait0 = _sig("semkv_set_first_copy_wait_polls", None, [_i32])
+_lib_rcp_check = _sig("semkv_check_reciprocal", _i32, [_u32, _u32, _p, _p])
 _lib_score_ws = _sig("semkv_score_workspace_size", _sz, [_i32, _i32, _i32, _i32, _i32, _i32])
 _lib_score = _sig("semkv_score", _i32, [_i32, _p, _i64, _p, _p, _i32, _i32, _i32, _i32, _i32, _i32,
                                         _p, _p, _sz, _p, _p])
@@ -74,7 +75,7 @@ _lib_decode_acc = _sig("semkv_decode_attn_acc", _i32, [ctypes.POINTER(SemkvCache
 
 EXPORTED = ["semkv_num_high", "semkv_digits_per_word", "semkv_words_per_row", "semkv_row_bits",
             "semkv_pool_words", "semkv_version",
-            "semkv_set_first_copy_wait_polls",
+            "semkv_set_first_copy_wait_polls", "semkv_check_reciprocal",
             "semkv_score_workspace_size", "semkv_score", "semkv_select_workspace_size", "semkv_select",
             "semkv_quantize_workspace_size", "semkv_quantize", "semkv_quantize_noalloc",
             "semkv_append_workspace_size",
@@ -131,6 +132,13 @@ def semkv_version() -> str:
 def semkv_set_first_copy_wait_polls(polls: int) -> None:
     """Testing aid: poll bound of the first copy wait of later quantize/decode launches (< 0: default)."""
     _lib_set_wait0(int(polls))
+
+
+def semkv_check_reciprocal(exp_lo: int, exp_hi: int, stream=None) -> int:
+    """Differences between the quantizer's reciprocal and the IEEE one over exponent fields [exp_lo, exp_hi]."""
+    out = torch.zeros(1, dtype=torch.int64, device="cuda")
+    _check(_lib_rcp_check(exp_lo, exp_hi, _ptr(out), _stream(stream)), "semkv_check_reciprocal")
+    return int(out.item())
 
 
 # ------------------------------------------------------------------ a1 score

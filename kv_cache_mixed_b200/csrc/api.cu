@@ -162,6 +162,11 @@ const char *semkv_version(void) { return "semkv-b200 0.3 (sm_100a)"; }
 
 void semkv_set_first_copy_wait_polls(int32_t polls) { g_first_wait_polls = polls < 0 ? -1 : polls; }
 
+semkv_status semkv_check_reciprocal(uint32_t exp_lo, uint32_t exp_hi, unsigned long long *mismatches, void *stream) {
+  if (exp_lo < 1 || exp_hi > 254 || exp_lo > exp_hi || mismatches == nullptr) return SEMKV_ERR_INVALID_ARG;
+  return cuda_status(launch_reciprocal_check(exp_lo, exp_hi, mismatches, S(stream)));
+}
+
 size_t semkv_score_workspace_size(int32_t kind, int32_t B, int32_t T_max, int32_t H, int32_t H_q,
                                   int32_t w) {
   if (kind != SEMKV_SCORE_ATTN_MASS) return 0;

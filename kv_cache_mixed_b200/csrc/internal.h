@@ -28,6 +28,7 @@ cudaError_t encode_tensor_map_f16(CUtensorMap *map, const void *base, int rank, 
 
 // Slot of each token within its class, and the high count per sequence.
 //   slot int32 [B][T_max], cnt_high int32 [B].
+cudaError_t launch_reciprocal_check(uint32_t e_lo, uint32_t e_hi, unsigned long long *mismatches, cudaStream_t st);
 cudaError_t launch_slot_scan(const uint8_t *mask, int64_t mask_bstride, const int32_t *seq_len,
                              int len_const, int B, int T_max, const int32_t *n_high, const int32_t *n_low,
                              int32_t *slot, int32_t *cnt_high, uint32_t *status, cudaStream_t st);
