@@ -229,6 +229,19 @@ __device__ __forceinline__ void f16_floor_steps(uint32_t xb, uint32_t (&out)[NR]
   }
 }
 
+// floor(x / D) for any 32-bit x, on the fp64 pipe instead of a 32-bit
+// multiply-high: x is exact as the double 2^52 + x minus 2^52, inv >= 1/D is
+// within 2^-49 of it (relative), so x * inv exceeds x / D by less than 1/D and
+// one fma rounded toward zero onto 2^52 (unit last place 1) leaves
+// floor(x / D) in the low word.  The integer pipe that the rest of the
+// digit extraction loads is spared the word's widest multiply.
+template <uint32_t D>
+__device__ __forceinline__ uint32_t div_fp64(uint32_t x) {
+  constexpr double inv = (1.0 / (double)D) * (1.0 + 0x1p-50);
+  const double xd = __hiloint2double(0x43300000, (int)x) - 4503599627370496.0;
+  return (uint32_t)__double2loint(__fma_rz(xd, inv, 4503599627370496.0));
+}
+
 // register pair J of a word (parts 2J, 2J+1) and the ones after it: the
 // parts' floors (keys) or their digits (values); `rest` holds the
 // word's digits from part 2J on
@@ -239,7 +252,7 @@ __device__ __forceinline__ void extract_regs(uint32_t rest, uint32_t (&out)[NR],
     uint32_t v = rest, next = 0;
     if constexpr (J < plan_regs(L) - 1) {
       constexpr uint32_t D = (uint32_t)ipow(L, ka + kb);
-      next = rest / D;
+      next = div_fp64<D>(rest);
       v = rest - next * D;
     }
     uint32_t xb;

@@ -122,3 +122,32 @@ def test_floor_coefficients_recover_the_digit_dot_product():
         d = np.stack([(P // L ** s) % L for s in range(k)], 1)
         x = np.stack([P // L ** s for s in range(k)], 1)
         assert np.allclose(d @ q, x @ coef, rtol=0, atol=1e-9)
+
+
+def _fp64_floor_div(x, D):
+    """decode.cu div_fp64<D>: x as an exact double, inv = RN(RN(1/D) * RN(1 + 2^-50)) (IEEE double, as
+    the constant is folded), then fma(x, inv, 2^52) rounded toward zero; the low word is floor(x * inv)."""
+    from fractions import Fraction
+    inv = (1.0 / D) * (1.0 + 2.0 ** -50)
+    return int(Fraction(x) * Fraction(inv)) , inv
+
+
+@pytest.mark.parametrize("L", [L for L in range(3, 16) if L not in (4, 8)])
+def test_fp64_word_split_is_floor_division(L):
+    # the word's first split divides by L^(p0 + p1), p0 and p1 the first two parts of the plan
+    from fractions import Fraction
+    parts, _ = _plans()[L]
+    n = O.digits_per_word(L)
+    divisors = {L ** (parts[2 * j] + parts[2 * j + 1]) for j in range((len(parts) - 1) // 2)} | \
+               {L ** k for k in range(1, n + 1) if L ** k < 2 ** 32}
+    rng = np.random.default_rng(L)
+    for D in sorted(divisors):
+        _, inv = _fp64_floor_div(0, D)
+        # inv bounds 1/D from above, closely enough that x * inv never reaches the next integer
+        assert Fraction(inv) >= Fraction(1, D)
+        assert (2 ** 32) * (Fraction(inv) - Fraction(1, D)) * D < 1
+        xs = [0, 1, D - 1, D, L ** n - 1, 2 ** 32 - 1] + [m * D + e for m in (1, 7, (2 ** 32 - 1) // D)
+                                                        for e in (-1, 0, 1) if 0 <= m * D + e < 2 ** 32]
+        xs += [int(v) for v in rng.integers(0, 2 ** 32, 200)]
+        for x in xs:
+            assert _fp64_floor_div(x, D)[0] == x // D, (L, D, x)
