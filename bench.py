@@ -48,12 +48,12 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 # kernels one default step launches: attention-mass score 4 (pass 1, merge,
-# pass 2, head sum), select 1, quantize 3 (slot scan, quantize+pack, count
-# advance), append 1, decode 3 (both pools in one launch -- every level pair the
-# workloads use has a merged instance --, FP16 block, merge)
-LAUNCHES_PER_STEP = 4 + 1 + 3 + 1 + 3
+# pass 2, head sum), select 1, quantize 2 (slot scan with the count advance,
+# quantize+pack), append 1, decode 3 (both pools in one launch -- every level
+# pair the workloads use has a merged instance --, FP16 block, merge)
+LAUNCHES_PER_STEP = 4 + 1 + 2 + 1 + 3
 DECODE_LAUNCHES = 3
-QUANT_LAUNCHES = 3
+QUANT_LAUNCHES = 2
 METRIC = "KV quantize+pack GB/s (FP16 in) & mixed-prec decode-attn GB/s vs HBM roofline"
 KERNEL_SOURCES = ["kv_cache_mixed_b200/csrc/quantize.cu", "kv_cache_mixed_b200/csrc/common.cuh"]
 DECODE_SOURCES = ["kv_cache_mixed_b200/csrc/decode.cu", "kv_cache_mixed_b200/csrc/common.cuh"]

@@ -69,7 +69,7 @@ semkv_status quantize_rows(semkv_cache *c, const uint16_t *k, const uint16_t *v,
   int32_t *slot = reinterpret_cast<int32_t *>(ws);
   int32_t *cnt = reinterpret_cast<int32_t *>(reinterpret_cast<char *>(ws) + up256((size_t)c->B * T_stride * 4));
   cudaError_t e = launch_slot_scan(mask, mask_bstride, seq_len, len_const, c->B, T_stride, c->n_high, c->n_low,
-                                   slot, cnt, status, st);
+                                   c->cap_high, c->cap_low, slot, cnt, status, st);
   if (e != cudaSuccess) return SEMKV_ERR_CUDA;
   QuantLaunch q;
   q.k = k;
@@ -83,7 +83,6 @@ semkv_status quantize_rows(semkv_cache *c, const uint16_t *k, const uint16_t *v,
   q.mask = mask;
   q.mask_bstride = mask_bstride;
   q.slot = slot;
-  q.cnt_high = cnt;
   q.n_high = c->n_high;
   q.n_low = c->n_low;
   q.k_high = c->k_high;

@@ -26,12 +26,13 @@ cudaError_t kernel_occupancy(const void *fn, int threads, int smem_bytes, int *c
 cudaError_t encode_tensor_map_f16(CUtensorMap *map, const void *base, int rank, const uint64_t *dims,
                                   const uint64_t *strides_bytes, const uint32_t *box, bool swizzle128);
 
-// Slot of each token within its class, and the high count per sequence.
+// Slot of each token within its class and the high count per sequence, then
+// the per-sequence counts advanced (clamped to the capacities).
 //   slot int32 [B][T_max], cnt_high int32 [B].
 cudaError_t launch_reciprocal_check(uint32_t e_lo, uint32_t e_hi, unsigned long long *mismatches, cudaStream_t st);
 cudaError_t launch_slot_scan(const uint8_t *mask, int64_t mask_bstride, const int32_t *seq_len,
-                             int len_const, int B, int T_max, const int32_t *n_high, const int32_t *n_low,
-                             int32_t *slot, int32_t *cnt_high, uint32_t *status, cudaStream_t st);
+                             int len_const, int B, int T_max, int32_t *n_high, int32_t *n_low, int cap_high,
+                             int cap_low, int32_t *slot, int32_t *cnt_high, uint32_t *status, cudaStream_t st);
 
 struct QuantLaunch {
   const uint16_t *k, *v;            // [B][Lyr][H][T_stride][128]
@@ -41,7 +42,6 @@ struct QuantLaunch {
   const uint8_t *mask;
   int64_t mask_bstride;
   const int32_t *slot;              // [B][T_stride]
-  const int32_t *cnt_high;          // [B]
   int32_t *n_high, *n_low;          // device counts (bases before, advanced after)
   uint32_t *k_high, *v_high, *k_low, *v_low;
   float *k_high_meta, *v_high_meta, *k_low_meta, *v_low_meta;
