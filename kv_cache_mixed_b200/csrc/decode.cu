@@ -932,6 +932,8 @@ __device__ __forceinline__ void pool_body(const DecParams &p, const PoolArgs &pa
 template <int LA, int LB, bool ROT, bool PAGES, bool WIDE>
 __global__ void __launch_bounds__(DEC_WARPS * 32, 4) decode_pool_kernel(const DecParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
+  // the FP16-block kernel after it reads nothing this kernel writes: let it start
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int n0 = p.slabs * p.pool[0].S;
   const int cls = (int)blockIdx.x >= n0;
   const int i = cls ? (int)blockIdx.x - n0 : (int)blockIdx.x;
@@ -1035,6 +1037,10 @@ __global__ void __launch_bounds__(128) decode_buffer_kernel(const BufParams p) {
       dst[qh * PART_STRIDE + 1] = n > 0 ? red[qh][1] : 0.0f;
     }
   }
+  // Launched as a dependent of the pool kernel, it may run alongside it; it
+  // finishes only after the pool kernel has, so the merge kernel that waits
+  // for it sees both kernels' partials.  (Every thread gets here.)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 // ---- merge all partials of a (sequence, layer, KV head) for one query head:
@@ -1304,11 +1310,13 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int sc
                         reinterpret_cast<const float2 *>(c.v_low_meta), c.n_low, c.cap_low, Sl, Sh,
                         slab_words(c, c.L_low, c.cap_low)};
   cudaError_t e;
+  bool pool_launched = false;          // the last launch so far is a pool kernel
   if (has_merged(c.L_high, c.L_low)) {
     p.pool[0] = high;
     p.pool[1] = low;
     e = launch_classes(true, c.L_high, c.L_low, c, p, slabs * (Sh + Sl), st);
     if (e != cudaSuccess) return e;
+    pool_launched = slabs * (Sh + Sl) > 0;
   } else {
     for (int cls = 0; cls < 2; ++cls) {
       p.pool[0] = cls ? low : high;
@@ -1317,6 +1325,7 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int sc
       const int L = cls ? c.L_low : c.L_high;
       e = launch_classes(false, L, L, c, p, slabs * p.pool[0].S, st);
       if (e != cudaSuccess) return e;
+      pool_launched = pool_launched || slabs * p.pool[0].S > 0;
     }
   }
   // FP16 block
@@ -1333,8 +1342,26 @@ cudaError_t launch_decode(const semkv_cache &c, int layer0, int n_layers, int sc
   float *prob = logit + (size_t)c.B * c.H_q * c.block;
   bp.score_li = score_li;
   bp.logit = logit;
-  decode_buffer_kernel<<<slabs, 128, 0, st>>>(bp);
-  e = cudaGetLastError();
+  if (pool_launched) {
+    // programmatic dependent launch right behind a pool kernel: the FP16-block
+    // kernel reads only the block, q and its own outputs, so it may overlap the
+    // pool kernel; it waits for that kernel before it exits.  (Behind any
+    // other launch it must not start early: the block may still be written.)
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(slabs);
+    cfg.blockDim = dim3(128);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_buffer_kernel, bp);
+  } else {
+    decode_buffer_kernel<<<slabs, 128, 0, st>>>(bp);
+    e = cudaGetLastError();
+  }
   if (e != cudaSuccess) return e;
   MergeAcc ma;
   ma.rot = c.rotate;
